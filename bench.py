@@ -1,0 +1,402 @@
+#!/usr/bin/env python
+"""Benchmark: one sparse MoE layer forward pass on B200 (gpt-oss-120b-shaped decode).
+
+Workload: d_model=2880, 128 experts, top-4, SwiGLU d_ff=2880, MXFP4 expert
+weights (E2M1 + E8M0 per 32), bf16 router and activations, T=64 tokens per
+step (the largest decode batch of the configuration; seeded synthetic inputs).
+A step is one moe_layer_forward: router, top-k, permutation, grouped SwiGLU
+FFN over the routed experts, combine.
+
+    python bench.py [--gpus N --steps K --warmup W] [--tokens T] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs its own batch on
+its own GPU (independent decode batches; no data-path collective), times are
+the max over ranks, and ``value`` is all ranks' tokens per second.
+``--impl reference`` times the fp64 CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import moe_inputs as mi  # noqa: E402
+
+METRIC = "MoE-layer tokens/s and achieved HBM GB/s (decode) / TFLOPS (prefill) vs B200 peak"
+SHAPE = mi.GPTOSS
+L2_BYTES = 126 * 2 ** 20
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "src": "measured"}
+    return {"hbm_gbs": 6650.0, "src": "fallback"}
+
+
+def expert_bytes_split(shape):
+    """(W13 bytes, W2 bytes) of one expert, codes + scales."""
+    d, f = shape.d_model, shape.d_ff
+    blk = mi.BLOCK[shape.wdtype]
+    sb = {"mxfp4": 1, "nvfp4": 1, "int4": 2}.get(shape.wdtype, 0)
+    if shape.wdtype == "bf16":
+        return 2 * f * d * 2, d * f * 2
+    return 2 * f * d // 2 + 2 * f * (d // blk) * sb, d * f // 2 + d * (f // blk) * sb
+
+
+def workload_name(shape, T):
+    return (f"{shape.name}: d_model={shape.d_model} E={shape.n_experts} top-{shape.top_k} "
+            f"d_ff={shape.d_ff} {shape.wdtype.upper()} experts, T={T} tokens/step")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of the GPU's SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id: str):
+        self.bus_id = bus_id.lower()
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 10:
+                continue
+            if self.bus_id and not parts[1].lower().endswith(self.bus_id[-12:]):
+                continue
+            rows.append(parts)
+        if not rows:
+            return None
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# --------------------------------------------------------------- oracle leg
+def oracle_subset_layer(dlay, tokens):
+    """A host layer holding x/router/bias and only the experts the given tokens need."""
+    import torch
+    from oracle import layer as OL
+    hl = {"shape": dlay["shape"], "x": dlay["x"].cpu(), "router": dlay["router"].cpu(),
+          "bias": dlay["bias"].cpu() if dlay.get("bias") is not None else None, "shared": None}
+    logits = OL.router_logits(OL.to_f64(hl["x"])[tokens], OL.to_f64(hl["router"]),
+                              OL.to_f64(hl["bias"]) if hl["bias"] is not None else None)
+    idx, _, _ = OL.topk_select(logits, dlay["shape"].top_k)
+    need = sorted(set(idx.reshape(-1).tolist()))
+
+    class Lazy:
+        def __init__(self, src):
+            self.cache = {e: src[e].cpu() for e in need}
+
+        def __getitem__(self, e):
+            return self.cache[int(e)]
+
+    hl["experts"] = {k: Lazy(v) for k, v in dlay["experts"].items()}
+    if dlay.get("shared"):
+        hl["shared"] = {k: v.cpu() for k, v in dlay["shared"].items()}
+    _ = torch
+    return hl, need
+
+
+def time_oracle(hl, tokens):
+    from oracle import layer as OL
+    t0 = time.perf_counter()
+    OL.moe_layer(hl, tokens=tokens)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(dlay, T, budget_s=15.0):
+    """Oracle tokens/s on a bounded sample of the batch, single BLAS thread."""
+    try:
+        from threadpoolctl import threadpool_limits
+    except Exception:  # pragma: no cover
+        threadpool_limits = None
+    ctx = threadpool_limits(limits=1) if threadpool_limits else None
+    try:
+        hl, _ = oracle_subset_layer(dlay, [0])
+        t1 = time_oracle(hl, [0])
+        n = int(max(1, min(T, budget_s / max(t1, 1e-3))))
+        toks = list(range(n))
+        hl, need = oracle_subset_layer(dlay, toks)
+        el = time_oracle(hl, toks)
+    finally:
+        if ctx is not None:
+            ctx.__exit__(None, None, None)
+    return {"value": n / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} of the {T} tokens of one batch ({len(need)} distinct experts decoded in fp64), "
+                      f"{el:.1f} s, numpy float64 with one BLAS thread"}
+
+
+# ------------------------------------------------------------- reference arm
+def run_reference(args):
+    """The fp64 oracle on the host cores, same workload and metric.  Each step is
+    one token of the batch (the oracle's smallest unit of this workload); the
+    number of timed steps is capped so the run ends within MOE_REF_BUDGET_S
+    seconds (default 150), and the line reports how many were timed."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    from threadpoolctl import threadpool_limits
+    T = args.tokens
+    shape = SHAPE
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    budget = float(os.environ.get("MOE_REF_BUDGET_S", "150"))
+    t_draw = time.perf_counter()
+    dlay = mi.draw_layer(shape, T, seed=1000, device=dev)  # the same inputs as the GPU arm
+    hl, need = oracle_subset_layer(dlay, list(range(T)))
+    del dlay
+    t_draw = time.perf_counter() - t_draw
+    from oracle import layer as OL
+    order = list(range(T))
+    with threadpool_limits(limits=1):
+        n_warm = 0
+        t_step = None
+        for s in range(args.warmup):
+            t0 = time.perf_counter()
+            OL.moe_layer(hl, tokens=[order[s % T]])
+            t_step = time.perf_counter() - t0
+            n_warm += 1
+            if t_step * (s + 2) > budget / 4:
+                break
+        n = args.steps
+        if t_step is not None:
+            n = int(max(3, min(args.steps, (budget - n_warm * t_step) / t_step)))
+        t0 = time.perf_counter()
+        for s in range(n):
+            OL.moe_layer(hl, tokens=[order[(n_warm + s) % T]])
+        el = time.perf_counter() - t0
+    value = n / el
+    sample = (f"each step: 1 token of the T={T} batch through the fp64 oracle (router, top-k, "
+              f"{shape.top_k} MXFP4 experts decoded to fp64, SwiGLU, combine); numpy, one BLAS thread; "
+              f"{n} timed steps of {args.steps} requested (time budget {budget:.0f} s)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": n, "steps_requested": args.steps, "warmup": n_warm, "ms_per_step": 1000 * el / n,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_name(shape, T), "tokens": T, "input_setup_s": round(t_draw, 1)},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- our arm
+def kernel_src_sha():
+    p = os.path.join(ROOT, "expert_ffn_layer_route_b200", "csrc", "ffn_stream.cu")
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def stored_traffic(T):
+    """DRAM bytes per launch of the stage-1 kernel from a committed ncu summary,
+    if it was taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "ffn_stream_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    ent = d.get(f"gptoss_decode_T{T}")
+    if not ent or ent.get("kernel_src_sha") != kernel_src_sha():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import expert_ffn_layer_route_b200 as moe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    T = args.tokens
+    shape = SHAPE
+    dlay = mi.draw_layer(shape, T, seed=1000 + rank, device=dev)
+    desc = moe.make_desc(shape, T)
+    ws = torch.empty(moe.moe_workspace_size(desc), dtype=torch.uint8, device=dev)
+    out = torch.empty(T, shape.d_model, dtype=torch.bfloat16, device=dev)
+    routed = moe.make_weights(dlay["experts"])
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        moe.moe_layer_forward(desc, dlay["x"], dlay["router"], None, routed, None, out, ws, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    # routing of this batch -> algorithmic bytes
+    L = moe.moe_workspace_layout_of(desc)
+    offs = ws[L.offsets: L.offsets + 4 * (shape.n_experts + 1)].view(torch.int32).cpu().numpy()
+    distinct = int((np.diff(offs) > 0).sum())
+    b13, b2 = expert_bytes_split(shape)
+    act_bytes = 2 * T * shape.d_model * 2
+    router_bytes = shape.n_experts * shape.d_model * 2
+    layer_bytes = distinct * (b13 + b2) + router_bytes + act_bytes
+    stage1_bytes = distinct * b13 + T * shape.d_model * 2 + T * shape.top_k * shape.d_ff * 2
+
+    moe.moe_profile_enable(True)
+    moe.moe_profile_collect()
+    bus = ""
+    try:
+        bus = torch.cuda.get_device_properties(dev).pci_bus_id
+    except Exception:
+        pass
+    clocks = ClockSampler(bus) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop() if clocks else None
+    moe.moe_profile_enable(False)
+    prof = moe.moe_profile_collect()
+    ms = e0.elapsed_time(e1)
+    t_max = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    ms = float(t_max.item())
+    launches = int(sum(v[0] for v in prof.values()))
+
+    # end to end: pinned host input -> device, layer, result -> pinned host, every step
+    xh = dlay["x"].cpu().pin_memory()
+    oh = torch.empty(T, shape.d_model, dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty_like(dlay["x"])
+
+    def e2e_step():
+        xd.copy_(xh, non_blocking=True)
+        moe.moe_layer_forward(desc, xd, dlay["router"], None, routed, None, out, ws, stream)
+        oh.copy_(out, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2 = torch.cuda.Event(enable_timing=True)
+    e3 = torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e3.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms_e2e = torch.tensor([e2.elapsed_time(e3)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_e2e, op=dist.ReduceOp.MAX)
+    ms_e2e = float(ms_e2e.item())
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(dlay, T)
+
+    if rank == 0:
+        pk = peaks()
+        s1 = prof.get("ffn_stage1_gate_up", (0, 0.0))
+        s1_ms = s1[1] / max(s1[0], 1)
+        achieved = stage1_bytes / (s1_ms * 1e-3) / 1e9 if s1_ms else 0.0
+        traffic = stored_traffic(T)
+        per_kernel = {k: {"launches": v[0], "avg_us": 1000.0 * v[1] / max(v[0], 1),
+                          "share": v[1] / max(sum(w[1] for w in prof.values()), 1e-12)} for k, v in prof.items()}
+        value = world * T * args.steps / (ms * 1e-3)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": workload_name(shape, T), "tokens": T, "weights": "mxfp4",
+                       "parallelism": f"replicas x{world} (independent decode batches)",
+                       "l2": f"inputs larger than L2: {distinct} distinct experts = "
+                             f"{distinct * (b13 + b2) / 1e9:.2f} GB of weights per step vs {L2_BYTES / 2**20:.0f} MiB L2",
+                       "distinct_experts": distinct, "layer_algorithmic_bytes": layer_bytes,
+                       "layer_achieved_gbs": layer_bytes / (ms / args.steps * 1e-3) / 1e9},
+            "roofline": {"bound": "hbm", "kernel": "ffn_stage1_gate_up", "achieved": achieved,
+                         "peak": pk["hbm_gbs"], "peak_source": pk["src"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                         "algorithmic_bytes_per_launch": stage1_bytes, "avg_launch_us": 1000 * s1_ms},
+            "kernels": per_kernel,
+            "gpu_launches": launches,
+            "e2e": {"value": world * T * args.steps / (ms_e2e * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": T * shape.d_model * 2, "d2h_bytes_per_step": T * shape.d_model * 2},
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--tokens", type=int, default=64)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,232 @@
+// Shared device helpers for the MoE layer kernels (sm_100a).
+//
+// Inline-PTX wrappers for mbarriers, 1-D bulk copies (cp.async.bulk), the
+// legacy warp-level tensor-core MMA used by the decode path, fp4 -> fp16
+// conversion, and the bounded waits every kernel uses instead of unbounded
+// spins.  A wait that runs out records MOE_ERR_TIMEOUT in the library's device
+// status word and returns false; it never traps.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// Sticky device status word (first error wins).  Defined in moe_api.cu.
+extern __device__ int g_status;
+
+__device__ __forceinline__ void set_status(int code) { atomicCAS(&g_status, 0, code); }
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Limit for any single device-side wait.  Every legitimate wait in these
+// kernels ends within microseconds; two seconds only guards against a bug.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// ---------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity to complete.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      set_status(MOE_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// -------------------------------------------------------------- bulk copy
+// L2 policy for streamed-once weights.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completing `bytes` on `bar`.
+// dst/src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                              uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], "
+      "%4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// ------------------------------------------------------------ smem loads
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds8(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+
+// ------------------------------------------------------------------- MMA
+// D = A(16x16, row) * B(16x8, col) + C, fp32 accumulate.
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ------------------------------------------------------ format conversion
+// Four packed E2M1 pairs (one 32-bit word = 8 codes) -> four f16x2 words.
+// Output i holds the codes of byte i: low nibble in the low half.
+__device__ __forceinline__ void e2m1x8_to_f16x8(uint32_t w, uint32_t& o0, uint32_t& o1, uint32_t& o2,
+                                                uint32_t& o3) {
+  asm("{\n .reg .b8 q0, q1, q2, q3;\n mov.b32 {q0, q1, q2, q3}, %4;\n"
+      " cvt.rn.f16x2.e2m1x2 %0, q0;\n cvt.rn.f16x2.e2m1x2 %1, q1;\n"
+      " cvt.rn.f16x2.e2m1x2 %2, q2;\n cvt.rn.f16x2.e2m1x2 %3, q3;\n}\n"
+      : "=r"(o0), "=r"(o1), "=r"(o2), "=r"(o3)
+      : "r"(w));
+}
+
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+  __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// E8M0 byte -> fp32 2^(v-127) (v = 255 -> NaN).
+__device__ __forceinline__ float e8m0_to_f32(uint32_t v) {
+  if (v == 0u) return __int_as_float(0x00400000);  // 2^-127 (subnormal)
+  if (v == 255u) return __int_as_float(0x7fc00000);
+  return __int_as_float(static_cast<int>(v << 23));
+}
+
+// E4M3 (FN) byte -> fp16 bits (exact: every finite E4M3 value is an fp16 value).
+__device__ __forceinline__ uint16_t e4m3_to_f16_bits(uint32_t b) {
+  const uint32_t s = (b >> 7) & 1u, e = (b >> 3) & 15u, m = b & 7u;
+  if (e == 15u && m == 7u) return 0x7e00u;  // NaN
+  uint32_t h;
+  if (e == 0u) {
+    // subnormal m/8 * 2^-6 = m * 2^-9 ; in fp16 that is a normal number for m>0
+    if (m == 0u) {
+      h = 0u;
+    } else {
+      // normalise: value = m * 2^-9, m in 1..7
+      int lz = __clz(m) - 29;           // leading zeros within 3 bits
+      uint32_t mm = (m << (lz + 1)) & 7u; // drop the leading one
+      int ex = -9 + (2 - lz);            // exponent of the leading one
+      h = (static_cast<uint32_t>(ex + 15) << 10) | (mm << 7);
+    }
+  } else {
+    h = ((e - 7u + 15u) << 10) | (m << 7);
+  }
+  return static_cast<uint16_t>((s << 15) | h);
+}
+
+// 8 INT4 codes (two's complement, one 32-bit word) -> four f16x2 words holding
+// exactly the integers q in [-8, 7].  Pairing: o0 = (n0, n4), o1 = (n1, n5),
+// o2 = (n2, n6), o3 = (n3, n7), where nI is nibble I counting from bit 0.
+// Uses f16 1024 + u (u = q + 8 in the mantissa) and subtracts 1032.
+__device__ __forceinline__ void int4x8_to_f16x8(uint32_t w, uint32_t& o0, uint32_t& o1, uint32_t& o2,
+                                                uint32_t& o3) {
+  const uint32_t u = w ^ 0x88888888u;  // q + 8 per nibble
+  const uint32_t magic = 0x64006400u;  // f16 (1024, 1024)
+  const uint32_t lo0 = (u & 0x000f000fu) | magic;         // 1024 + u0, 1024 + u4
+  const uint32_t hi0 = (u & 0x00f000f0u) | magic;         // 1024 + 16 u1, ...
+  const uint32_t lo1 = ((u >> 8) & 0x000f000fu) | magic;  // u2, u6
+  const uint32_t hi1 = ((u >> 8) & 0x00f000f0u) | magic;  // 16 u3, 16 u7
+  const __half2 k1032 = __half2half2(__ushort_as_half(0x6408u));  // 1032
+  const __half2 k72 = __half2half2(__ushort_as_half(0x5480u));    // 72
+  const __half2 k16th = __half2half2(__ushort_as_half(0x2c00u));  // 1/16
+  __half2 r0 = __hsub2(*reinterpret_cast<const __half2*>(&lo0), k1032);
+  __half2 r1 = __hfma2(*reinterpret_cast<const __half2*>(&hi0), k16th, __hneg2(k72));
+  __half2 r2 = __hsub2(*reinterpret_cast<const __half2*>(&lo1), k1032);
+  __half2 r3 = __hfma2(*reinterpret_cast<const __half2*>(&hi1), k16th, __hneg2(k72));
+  o0 = *reinterpret_cast<uint32_t*>(&r0);
+  o1 = *reinterpret_cast<uint32_t*>(&r1);
+  o2 = *reinterpret_cast<uint32_t*>(&r2);
+  o3 = *reinterpret_cast<uint32_t*>(&r3);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __int_as_float(static_cast<int>(b << 16)); }
+
+__host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace moe

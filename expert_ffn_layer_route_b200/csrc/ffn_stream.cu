@@ -1,0 +1,548 @@
+// Grouped SwiGLU expert FFN, weight-streaming form (decode and small groups).
+//
+// During decode each new token reads the weights of its active experts
+// ("Mixture of experts VRAM: total vs active parameters", section "What
+// active parameters change"), and with a batch the tokens of one step go to
+// different experts, so a step touches many experts; grouping the tokens
+// that chose the same expert lets one weight read serve all of them
+// ("Understanding MoE Inference Costs on Galactus", section "Prompt
+// processing is a different phase").  This kernel therefore walks work items
+// (expert, row tile) and streams each tile's weight rows from HBM exactly once
+// per pass of up to 32 of the expert's rows, applying them to all of those
+// rows at once.  The expert's gate / up / down projections (FloE verdict
+// page, JSON field referee_report.summary) are applied as SwiGLU:
+//   stage 1: h = silu(x W_gate^T) * (x W_up^T)   (gate and up tiles paired)
+//   stage 2: y = h W_down^T
+//
+// Block = 8 consumer warps + 1 producer warp.  The producer issues 1-D bulk
+// copies (cp.async.bulk, completion on mbarriers) of 128-byte row chunks of
+// the tile's weight rows and of the matching activation rows into a ring of
+// shared-memory stages; consumers decode the 4-bit codes to fp16 (E2M1 with
+// the hardware cvt, INT4 by the 1024-offset trick), and run m16n8k16 MMAs
+// with fp32 accumulation.  Block scales: MXFP4 (E8M0 per 32) and INT4 (bf16
+// per 128) multiply the fp32 partial sums of their block; NVFP4 (E4M3 per 16)
+// multiplies the fp16 weights (the product is exact in fp16) and its fp32
+// global scale is applied in the epilogue.  Within each 32-wide K block lane
+// c of a quad holds K = 8c..8c+7, i.e. the MMA's K order is a fixed
+// permutation of the block, applied identically to both operands.
+#include "ffn_stream.cuh"
+#include "profile.cuh"
+
+namespace moe {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kRowsPerTile = 256;     // smem weight rows per item
+constexpr int kChunkBytes = 128;      // bytes of one weight row per stage
+constexpr int kMaxStages = 8;
+
+template <int F>
+struct FmtTraits;
+template <>
+struct FmtTraits<kBF16> {
+  static constexpr int kc = 64;       // K values per stage
+  static constexpr int sw = 192;      // smem weight row stride (bytes)
+  static constexpr int blk = 0;       // scale block (0: none)
+  static constexpr int sbytes = 0;    // bytes per scale
+};
+template <>
+struct FmtTraits<kMXFP4> {
+  static constexpr int kc = 256, sw = 144, blk = 32, sbytes = 1;
+};
+template <>
+struct FmtTraits<kNVFP4> {
+  static constexpr int kc = 256, sw = 144, blk = 16, sbytes = 1;
+};
+template <>
+struct FmtTraits<kINT4> {
+  static constexpr int kc = 256, sw = 144, blk = 128, sbytes = 2;
+};
+
+template <int F>
+__device__ __forceinline__ int scale_row_bytes(int K) {
+  return FmtTraits<F>::blk ? (K / FmtTraits<F>::blk) * FmtTraits<F>::sbytes : 0;
+}
+
+// Everything a block needs to know about one work item.
+struct Item {
+  int valid;
+  int shared_idx;   // >= 0 for a shared expert
+  int expert;       // logical expert (routed) or shared index
+  int tile;
+  int row_start;    // first routed row of the expert (routed), 0 for shared
+  int n_cols;       // rows of x this expert applies to
+  const uint8_t* wbase;
+  const uint8_t* sbase;
+  float gscale;
+};
+
+template <int F, bool kGateUp>
+__device__ __forceinline__ Item decode_item(const FfnArgs& a, int item, int ntile, int n_act, const int* act,
+                                            const int* offs) {
+  Item it{};
+  const int grp = item / ntile;
+  it.tile = item - grp * ntile;
+  it.valid = 1;
+  if (grp < a.n_shared) {
+    it.shared_idx = grp;
+    it.expert = grp;
+    it.row_start = 0;
+    it.n_cols = a.T;
+    it.wbase = a.w_sh + (int64_t)grp * a.stride_w_sh;
+    it.sbase = a.s_sh ? a.s_sh + (int64_t)grp * a.stride_s_sh : nullptr;
+    it.gscale = (F == kNVFP4 && a.gsc_sh) ? __ldg(a.gsc_sh + grp) : 1.f;
+  } else {
+    const int e = act[grp - a.n_shared];
+    it.shared_idx = -1;
+    it.expert = e;
+    it.row_start = offs[e];
+    it.n_cols = offs[e + 1] - offs[e];
+    int p = a.slot_map ? __ldg(a.slot_map + e) : e;
+    if (p == -1 && a.slot_map) {
+      it.valid = 0;  // not resident in this call: skipped
+      p = 0;
+    } else if (p < 0 || p >= a.n_phys || it.row_start < 0 || it.n_cols < 0 ||
+               it.row_start + it.n_cols > a.T * a.k) {
+      set_status(MOE_ERR_DEVICE_INDEX);
+      it.valid = 0;
+      p = 0;
+    }
+    it.wbase = a.w + (int64_t)p * a.stride_w;
+    it.sbase = a.s ? a.s + (int64_t)p * a.stride_s : nullptr;
+    it.gscale = (F == kNVFP4 && a.gsc) ? __ldg(a.gsc + e) : 1.f;
+  }
+  return it;
+}
+
+template <int F, int NG, bool kGateUp>
+__global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const FfnArgs a) {
+  using Tr = FmtTraits<F>;
+  constexpr int KC = Tr::kc;
+  constexpr int SW = Tr::sw;
+  constexpr int SX = KC * 2 + 64;           // smem activation row stride (bytes)
+  constexpr int XCOLS = NG * 8;             // activation rows per pass
+  constexpr int kBlocksPerChunk = KC / 32;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + kMaxStages;
+  uint64_t* sfull = empty + kMaxStages;
+  uint64_t* sempty = sfull + 2;
+  volatile int* s_abort = reinterpret_cast<volatile int*>(sempty + 2);
+  int* s_nact = reinterpret_cast<int*>(sempty + 2) + 1;
+  int* s_offs = reinterpret_cast<int*>(sempty + 2) + 4;  // [E+1]
+  int* s_act = s_offs + (a.E + 4);           // [E]
+  uint8_t* s_scale = smem + (((16 * kMaxStages + 32 + 16 + 8 * a.E + 64) + 127) & ~127);
+  uint8_t* s_stage = s_scale + a.n_scale_buf * a.smem_scale_bytes;
+  const int stage_w_bytes = kRowsPerTile * SW;
+  const int stage_bytes = stage_w_bytes + XCOLS * SX;
+
+  const int E = a.E;
+  // ---- block setup: barriers, routed-expert list
+  if (tid == 0) {
+    for (int i = 0; i < a.n_stages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kConsumerWarps);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sfull[i], 1);
+      mbar_init(&sempty[i], kConsumerWarps);
+    }
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  for (int i = tid; i <= E; i += kThreads) s_offs[i] = __ldg(a.offsets + i);
+  __syncthreads();
+  if (warp == 0) {
+    int n = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      const bool on = e < E && s_offs[e + 1] > s_offs[e];
+      const uint32_t m = __ballot_sync(0xffffffffu, on);
+      if (on) s_act[n + __popc(m & ((1u << lane) - 1u))] = e;
+      n += __popc(m);
+    }
+    if (lane == 0) *s_nact = n;
+  }
+  __syncthreads();
+  const int n_act = *s_nact;
+
+  const int rows_per_item = kGateUp ? kRowsPerTile / 2 : kRowsPerTile;
+  const int ntile = ceil_div(a.N, rows_per_item);
+  const int n_items = (a.n_shared + n_act) * ntile;
+  const int K = a.K;
+  const int row_bytes = (F == kBF16) ? K * 2 : K / 2;  // weight row bytes
+  const int srow = scale_row_bytes<F>(K);
+  const int nchunks = ceil_div(K, KC);
+  const int nstage = a.n_stages;
+  const int nsb = a.n_scale_buf;
+
+  if (warp == kConsumerWarps) {
+    // ===================================================== producer warp
+    const uint64_t pol = l2_evict_first_policy();
+    uint32_t cnt = 0;  // stages issued
+    int item_no = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++item_no) {
+      const Item it = decode_item<F, kGateUp>(a, item, ntile, n_act, s_act, s_offs);
+      const int r0 = it.tile * rows_per_item;
+      const int nrows = min(rows_per_item, a.N - r0);  // valid rows per half
+      const int passes = it.valid ? ceil_div(it.n_cols, XCOLS) : 0;
+      const int sb = item_no % nsb;
+      const uint32_t suse = item_no / nsb;
+      const int sc_at = (nsb == 2) ? 0 : min(nstage - 1, nchunks - 1);
+      for (int pass = 0; pass < max(passes, 1); ++pass) {
+        const int c0 = pass * XCOLS;
+        const int ncols = passes ? min(XCOLS, it.n_cols - c0) : 0;
+        for (int ch = 0; ch < nchunks; ++ch) {
+          if (Tr::blk && pass == 0 && ch == sc_at) {
+            // block scales of the item's rows (whole K), one or two contiguous runs
+            if (!mbar_wait(&sempty[sb], (suse & 1u) ^ 1u)) { *s_abort = 1; }
+            if (*s_abort) break;
+            if (lane == 0) {
+              const uint32_t bytes = (uint32_t)(nrows * srow);
+              mbar_arrive_expect_tx(&sfull[sb], it.valid ? bytes * (kGateUp ? 2u : 1u) : 0u);
+              if (it.valid) {
+                uint8_t* dst = s_scale + sb * a.smem_scale_bytes;
+                bulk_g2s(dst, it.sbase + (int64_t)r0 * srow, bytes, &sfull[sb]);
+                if (kGateUp)
+                  bulk_g2s(dst + rows_per_item * srow, it.sbase + (int64_t)(a.N + r0) * srow, bytes, &sfull[sb]);
+              }
+            }
+            __syncwarp();
+          }
+          const int s = cnt % nstage;
+          const uint32_t par = ((cnt / nstage) & 1u) ^ 1u;
+          if (!mbar_wait(&empty[s], par)) *s_abort = 1;
+          if (*s_abort) break;
+          const int kb = ch * kChunkBytes;  // byte offset of this chunk inside a weight row
+          const uint32_t wbytes = (uint32_t)min(kChunkBytes, row_bytes - kb);
+          const uint32_t xbytes = (uint32_t)(min(KC, K - ch * KC) * 2);
+          const int nw = it.valid ? (kGateUp ? 2 * nrows : nrows) : 0;
+          if (lane == 0) mbar_arrive_expect_tx(&full[s], nw * wbytes + ncols * xbytes);
+          __syncwarp();
+          uint8_t* sw_base = s_stage + s * stage_bytes;
+          for (int r = lane; r < nw; r += 32) {
+            int grow, srow_i;
+            if (kGateUp) {
+              const bool up = r >= nrows;
+              const int rr = up ? r - nrows : r;
+              grow = (up ? a.N : 0) + r0 + rr;
+              srow_i = (up ? rows_per_item : 0) + rr;
+            } else {
+              grow = r0 + r;
+              srow_i = r;
+            }
+            bulk_g2s_hint(sw_base + srow_i * SW, it.wbase + (int64_t)grow * row_bytes + kb, wbytes, &full[s], pol);
+          }
+          uint8_t* sx_base = sw_base + stage_w_bytes;
+          for (int j = lane; j < ncols; j += 32) {
+            int src;
+            if (kGateUp)
+              src = it.shared_idx >= 0 ? (c0 + j) : __ldg(a.row_token + it.row_start + c0 + j);
+            else
+              src = it.shared_idx >= 0 ? (a.T * a.k + it.shared_idx * a.T + c0 + j) : (it.row_start + c0 + j);
+            bulk_g2s(sx_base + j * SX, a.xsrc + ((int64_t)src * K + (int64_t)ch * KC) * 2, xbytes, &full[s]);
+          }
+          ++cnt;
+        }
+        if (*s_abort) break;
+      }
+      if (*s_abort) break;
+    }
+    // Let every copy this warp issued land before the block can exit.
+    if (lane == 0) {
+      const uint32_t first = cnt > (uint32_t)nstage ? cnt - nstage : 0;
+      for (uint32_t c = first; c < cnt; ++c) mbar_wait(&full[c % nstage], (c / nstage) & 1u);
+    }
+    return;
+  }
+
+  // ======================================================= consumer warps
+  const int g = lane >> 2, c = lane & 3;
+  uint32_t cnt = 0;
+  int item_no = 0;
+  const uint32_t stage0 = smem_u32(s_stage);
+  const uint32_t scale0 = smem_u32(s_scale);
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++item_no) {
+    const Item it = decode_item<F, kGateUp>(a, item, ntile, n_act, s_act, s_offs);
+    const int r0 = it.tile * rows_per_item;
+    const int nrows = min(rows_per_item, a.N - r0);
+    const int passes = it.valid ? ceil_div(it.n_cols, XCOLS) : 0;
+    const int sb = item_no % nsb;
+    const uint32_t suse = item_no / nsb;
+    // smem rows of this warp's two m16 tiles
+    const int m0 = kGateUp ? warp * 16 : warp * 32;
+    const int m1 = kGateUp ? rows_per_item + warp * 16 : warp * 32 + 16;
+    const bool active = it.valid && (kGateUp ? (warp * 16 < nrows) : (warp * 32 < nrows));
+    if (Tr::blk) {
+      if (!mbar_wait(&sfull[sb], suse & 1u)) *s_abort = 1;
+    }
+    const uint32_t sc_base = scale0 + sb * a.smem_scale_bytes;
+    for (int pass = 0; pass < max(passes, 1); ++pass) {
+      const int c0 = pass * XCOLS;
+      const int ncols = passes ? min(XCOLS, it.n_cols - c0) : 0;
+      const int ng_act = ceil_div(ncols, 8);
+      float acc[NG][2][4];
+#pragma unroll
+      for (int q = 0; q < NG; ++q)
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) acc[q][mt][r] = 0.f;
+      float tmp[NG][2][4];  // INT4 group partials
+      for (int ch = 0; ch < nchunks; ++ch) {
+        const int s = cnt % nstage;
+        if (!mbar_wait(&full[s], (cnt / nstage) & 1u)) *s_abort = 1;
+        if (*s_abort) break;
+        if (active && ncols > 0) {
+          const uint32_t wst = stage0 + s * stage_bytes;
+          const uint32_t xst = wst + stage_w_bytes;
+          const int nblk = min(KC, K - ch * KC) / 32;
+#pragma unroll 2
+          for (int b = 0; b < nblk; ++b) {
+            uint32_t A[2][2][4];  // [m-tile][k16 tile][reg]
+            if constexpr (F == kBF16) {
+#pragma unroll
+              for (int mt = 0; mt < 2; ++mt) {
+                const int mr = mt ? m1 : m0;
+                const uint4 lo = lds128(wst + (mr + g) * SW + b * 64 + 16 * c);
+                const uint4 hi = lds128(wst + (mr + g + 8) * SW + b * 64 + 16 * c);
+                A[mt][0][0] = lo.x; A[mt][0][1] = hi.x; A[mt][0][2] = lo.y; A[mt][0][3] = hi.y;
+                A[mt][1][0] = lo.z; A[mt][1][1] = hi.z; A[mt][1][2] = lo.w; A[mt][1][3] = hi.w;
+              }
+            } else {
+#pragma unroll
+              for (int mt = 0; mt < 2; ++mt) {
+                const int mr = mt ? m1 : m0;
+                const uint32_t wlo = lds32(wst + (mr + g) * SW + b * 16 + 4 * c);
+                const uint32_t whi = lds32(wst + (mr + g + 8) * SW + b * 16 + 4 * c);
+                uint32_t l0, l1, l2, l3, h0, h1, h2, h3;
+                if constexpr (F == kINT4) {
+                  int4x8_to_f16x8(wlo, l0, l1, l2, l3);
+                  int4x8_to_f16x8(whi, h0, h1, h2, h3);
+                } else {
+                  e2m1x8_to_f16x8(wlo, l0, l1, l2, l3);
+                  e2m1x8_to_f16x8(whi, h0, h1, h2, h3);
+                }
+                if constexpr (F == kNVFP4) {
+                  // this lane's 8 values share one 16-block per row
+                  const int nb = (ch * KC + b * 32 + 8 * c) >> 4;
+                  const uint32_t slo = e4m3_to_f16_bits(lds8(sc_base + (mr + g) * srow + nb));
+                  const uint32_t shi = e4m3_to_f16_bits(lds8(sc_base + (mr + g + 8) * srow + nb));
+                  const uint32_t slo2 = slo | (slo << 16), shi2 = shi | (shi << 16);
+                  l0 = hmul2_u32(l0, slo2); l1 = hmul2_u32(l1, slo2); l2 = hmul2_u32(l2, slo2); l3 = hmul2_u32(l3, slo2);
+                  h0 = hmul2_u32(h0, shi2); h1 = hmul2_u32(h1, shi2); h2 = hmul2_u32(h2, shi2); h3 = hmul2_u32(h3, shi2);
+                }
+                A[mt][0][0] = l0; A[mt][0][1] = h0; A[mt][0][2] = l1; A[mt][0][3] = h1;
+                A[mt][1][0] = l2; A[mt][1][1] = h2; A[mt][1][2] = l3; A[mt][1][3] = h3;
+              }
+            }
+            float sc[2][2];
+            if constexpr (F == kMXFP4) {
+              const int blk = (ch * KC) / 32 + b;
+#pragma unroll
+              for (int mt = 0; mt < 2; ++mt) {
+                const int mr = mt ? m1 : m0;
+                sc[mt][0] = e8m0_to_f32(lds8(sc_base + (mr + g) * srow + blk));
+                sc[mt][1] = e8m0_to_f32(lds8(sc_base + (mr + g + 8) * srow + blk));
+              }
+            }
+            const bool grp_first = (F == kINT4) && ((b & 3) == 0);
+            const bool grp_last = (F == kINT4) && (((b & 3) == 3) || (b == nblk - 1));
+            if constexpr (F == kINT4) {
+              if (grp_first) {
+#pragma unroll
+                for (int q = 0; q < NG; ++q)
+#pragma unroll
+                  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) tmp[q][mt][r] = 0.f;
+              }
+            }
+#pragma unroll
+            for (int q = 0; q < NG; ++q) {
+              if (q < ng_act) {
+                const uint4 xv = lds128(xst + (q * 8 + g) * SX + b * 64 + 16 * c);
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt) {
+                  if constexpr (F == kMXFP4) {
+                    float t4[4] = {0.f, 0.f, 0.f, 0.f};
+                    mma_f16(t4, A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
+                    mma_f16(t4, A[mt][1][0], A[mt][1][1], A[mt][1][2], A[mt][1][3], xv.z, xv.w);
+                    acc[q][mt][0] = fmaf(t4[0], sc[mt][0], acc[q][mt][0]);
+                    acc[q][mt][1] = fmaf(t4[1], sc[mt][0], acc[q][mt][1]);
+                    acc[q][mt][2] = fmaf(t4[2], sc[mt][1], acc[q][mt][2]);
+                    acc[q][mt][3] = fmaf(t4[3], sc[mt][1], acc[q][mt][3]);
+                  } else if constexpr (F == kINT4) {
+                    mma_f16(tmp[q][mt], A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
+                    mma_f16(tmp[q][mt], A[mt][1][0], A[mt][1][1], A[mt][1][2], A[mt][1][3], xv.z, xv.w);
+                  } else if constexpr (F == kNVFP4) {
+                    mma_f16(acc[q][mt], A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
+                    mma_f16(acc[q][mt], A[mt][1][0], A[mt][1][1], A[mt][1][2], A[mt][1][3], xv.z, xv.w);
+                  } else {
+                    mma_bf16(acc[q][mt], A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
+                    mma_bf16(acc[q][mt], A[mt][1][0], A[mt][1][1], A[mt][1][2], A[mt][1][3], xv.z, xv.w);
+                  }
+                }
+              }
+            }
+            if constexpr (F == kINT4) {
+              if (grp_last) {
+                const int grp = (ch * KC + b * 32) / 128;
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt) {
+                  const int mr = mt ? m1 : m0;
+                  const float s_lo = bf16_bits_to_f32(lds16(sc_base + (mr + g) * srow + 2 * grp));
+                  const float s_hi = bf16_bits_to_f32(lds16(sc_base + (mr + g + 8) * srow + 2 * grp));
+#pragma unroll
+                  for (int q = 0; q < NG; ++q) {
+                    acc[q][mt][0] = fmaf(tmp[q][mt][0], s_lo, acc[q][mt][0]);
+                    acc[q][mt][1] = fmaf(tmp[q][mt][1], s_lo, acc[q][mt][1]);
+                    acc[q][mt][2] = fmaf(tmp[q][mt][2], s_hi, acc[q][mt][2]);
+                    acc[q][mt][3] = fmaf(tmp[q][mt][3], s_hi, acc[q][mt][3]);
+                  }
+                }
+              }
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        ++cnt;
+      }
+      if (*s_abort) break;
+      // ---------------------------------------------------------- epilogue
+      if (active && ncols > 0) {
+#pragma unroll
+        for (int q = 0; q < NG; ++q) {
+          if (q < ng_act) {
+#pragma unroll
+            for (int hc = 0; hc < 2; ++hc) {
+              const int col = c0 + q * 8 + 2 * c + hc;
+              if (col < it.n_cols) {
+                float f = it.gscale;
+                if (F != kBF16) {
+                  int src;
+                  if (kGateUp)
+                    src = it.shared_idx >= 0 ? col : __ldg(a.row_token + it.row_start + col);
+                  else
+                    src = it.shared_idx >= 0 ? (a.T * a.k + it.shared_idx * a.T + col) : (it.row_start + col);
+                  f = ldexpf(f, __ldg(a.xexp + src));
+                }
+                if (kGateUp) {
+                  const int orow = it.shared_idx >= 0 ? (a.T * a.k + it.shared_idx * a.T + col) : (it.row_start + col);
+                  __nv_bfloat16* o = a.out_routed + (int64_t)orow * a.N + r0 + warp * 16;
+#pragma unroll
+                  for (int hr = 0; hr < 2; ++hr) {
+                    const float gt = acc[q][0][hr * 2 + hc] * f;
+                    const float up = acc[q][1][hr * 2 + hc] * f;
+                    const float h = gt / (1.f + expf(-gt)) * up;
+                    o[g + 8 * hr] = __float2bfloat16_rn(h);
+                  }
+                } else {
+                  __nv_bfloat16* o = it.shared_idx >= 0
+                                         ? a.out_shared + ((int64_t)it.shared_idx * a.T + col) * a.N
+                                         : a.out_routed + (int64_t)(it.row_start + col) * a.N;
+#pragma unroll
+                  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int hr = 0; hr < 2; ++hr)
+                      o[r0 + warp * 32 + mt * 16 + g + 8 * hr] = __float2bfloat16_rn(acc[q][mt][hr * 2 + hc] * f);
+                }
+              }
+            }
+          }
+        }
+      }
+    }
+    if (*s_abort) break;
+    if (Tr::blk) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sempty[sb]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host side
+struct FfnLaunch {
+  int F, NG;
+  bool gate_up;
+};
+
+template <int F, int NG, bool GU>
+static cudaError_t launch_one(const FfnArgs& a, int grid, size_t smem, cudaStream_t st) {
+  auto kern = ffn_stream_kernel<F, NG, GU>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  ProfScope prof(GU ? "ffn_stage1_gate_up" : "ffn_stage2_down", st);
+  kern<<<grid, kThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int F, bool GU>
+static cudaError_t dispatch_ng(const FfnArgs& a, int ng, int grid, size_t smem, cudaStream_t st) {
+  switch (ng) {
+    case 1: return launch_one<F, 1, GU>(a, grid, smem, st);
+    case 2: return launch_one<F, 2, GU>(a, grid, smem, st);
+    default: return launch_one<F, 4, GU>(a, grid, smem, st);
+  }
+}
+
+static int fmt_kc(int F) { return F == kBF16 ? 64 : 256; }
+static int fmt_sw(int F) { return F == kBF16 ? 192 : 144; }
+static int fmt_srow(int F, int K) {
+  switch (F) {
+    case kMXFP4: return K / 32;
+    case kNVFP4: return K / 16;
+    case kINT4: return (K / 128) * 2;
+    default: return 0;
+  }
+}
+
+// Shared memory plan of one stage kernel; returns false when it cannot fit.
+static bool plan_smem(int F, int ng, int K, int E, int smem_max, FfnArgs& a, size_t& total) {
+  const int hdr = ((16 * kMaxStages + 32 + 16 + 8 * E + 64) + 127) & ~127;
+  const int sbuf = ((kRowsPerTile * fmt_srow(F, K)) + 127) & ~127;
+  const int stage = kRowsPerTile * fmt_sw(F) + ng * 8 * (fmt_kc(F) * 2 + 64);
+  for (int nsb = 2; nsb >= 1; --nsb) {
+    if (F == kBF16 && nsb == 2) continue;
+    const int nsbx = (F == kBF16) ? 1 : nsb;
+    const int room = smem_max - hdr - nsbx * sbuf;
+    int ns = room / stage;
+    if (ns > kMaxStages) ns = kMaxStages;
+    if (ns >= 3 || (nsb == 1 && ns >= 2)) {
+      a.n_stages = ns;
+      a.n_scale_buf = nsbx;
+      a.smem_scale_bytes = sbuf;
+      total = (size_t)hdr + (size_t)nsbx * sbuf + (size_t)ns * stage;
+      return true;
+    }
+  }
+  return false;
+}
+
+cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, int T, int n_sms, int smem_max, cudaStream_t st,
+                              int* unsupported) {
+  *unsupported = 0;
+  const int ng = T <= 8 ? 1 : (T <= 16 ? 2 : 4);
+  size_t smem = 0;
+  if (!plan_smem(F, ng, a.K, a.E, smem_max, a, smem)) {
+    *unsupported = 1;
+    return cudaSuccess;
+  }
+  const int rows_per_item = gate_up ? kRowsPerTile / 2 : kRowsPerTile;
+  const int ntile = ceil_div(a.N, rows_per_item);
+  const long max_items = (long)(a.n_shared + (a.E < T * a.k ? a.E : T * a.k)) * ntile;
+  int grid = (int)(max_items < n_sms ? max_items : n_sms);
+  if (grid < 1) return cudaSuccess;
+  switch (F) {
+    case kBF16: return gate_up ? dispatch_ng<kBF16, true>(a, ng, grid, smem, st) : dispatch_ng<kBF16, false>(a, ng, grid, smem, st);
+    case kMXFP4: return gate_up ? dispatch_ng<kMXFP4, true>(a, ng, grid, smem, st) : dispatch_ng<kMXFP4, false>(a, ng, grid, smem, st);
+    case kNVFP4: return gate_up ? dispatch_ng<kNVFP4, true>(a, ng, grid, smem, st) : dispatch_ng<kNVFP4, false>(a, ng, grid, smem, st);
+    default: return gate_up ? dispatch_ng<kINT4, true>(a, ng, grid, smem, st) : dispatch_ng<kINT4, false>(a, ng, grid, smem, st);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,354 @@
+// C ABI entry points of the MoE layer library: argument checks, workspace
+// layout, and the order in which the kernels of one layer are enqueued.
+//
+// One layer call (page "Mixture of experts VRAM: total vs active parameters",
+// section "How current MoE models route each token": a router picks a few
+// experts per token; Galactus page, section "Prompt processing is a different
+// phase": tokens of one expert are grouped) runs, on the caller's stream:
+//   router logits -> top-k + gates -> stable permutation ->
+//   [4-bit: activation rows to fp16] -> stage 1 (gate/up + SwiGLU) ->
+//   [4-bit: h rows to fp16] -> stage 2 (down) -> weighted combine.
+// Nothing here allocates device memory; all scratch is carved from the
+// caller's workspace.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "ffn_stream.cuh"
+
+namespace moe {
+
+__device__ int g_status = 0;
+
+cudaError_t launch_route_topk(const moe_layer_desc& dsc, const void* x, const void* wr, const float* bias,
+                              float* logits, int32_t* topk_idx, float* topk_w, cudaStream_t st);
+cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* offsets, int32_t* row_token,
+                           int32_t* inv, cudaStream_t st);
+cudaError_t launch_prep_rows(const void* src, int rows, int K, bool perm_int4, void* dst, int32_t* rexp,
+                             cudaStream_t st);
+cudaError_t launch_combine(const void* y, const int32_t* inv, const float* gw, const void* y_shared, int n_shared,
+                           int T, int d, int k, void* out, cudaStream_t st);
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int fmt_block(int f) {
+  switch (f) {
+    case MOE_W_MXFP4: return 32;
+    case MOE_W_NVFP4: return 16;
+    case MOE_W_INT4_G128: return 128;
+    default: return 1;
+  }
+}
+int fmt_scale_bytes(int f) { return f == MOE_W_INT4_G128 ? 2 : (f == MOE_W_BF16 ? 0 : 1); }
+bool is4bit(int f) { return f != MOE_W_BF16; }
+
+// bytes of one [N][K] matrix's values / scales
+int64_t mat_bytes(int f, int64_t N, int64_t K) { return is4bit(f) ? N * K / 2 : N * K * 2; }
+int64_t scale_bytes(int f, int64_t N, int64_t K) {
+  return is4bit(f) ? N * (K / fmt_block(f)) * fmt_scale_bytes(f) : 0;
+}
+
+struct Layout {
+  size_t logits, topk_idx, topk_w, offsets, row_token, inv, xq, xexp, h, hq, hexp, y, ysh, total;
+};
+
+Layout layout_of(const moe_layer_desc& d) {
+  Layout L{};
+  const size_t T = d.T, E = d.n_experts, k = d.top_k, D = d.d_model, F = d.d_ff, S = d.n_shared;
+  const size_t R = T * k, RT = R + S * T;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o = align_up(o + bytes);
+    return at;
+  };
+  L.logits = take(T * E * 4);
+  L.topk_idx = take(T * k * 4);
+  L.topk_w = take(T * k * 4);
+  L.offsets = take((E + 1) * 4);
+  L.row_token = take(R * 4);
+  L.inv = take(R * 4);
+  const bool q = is4bit(d.wdtype);
+  L.xq = take(q ? T * D * 2 : 0);
+  L.xexp = take(q ? T * 4 : 0);
+  L.h = take(RT * F * 2);
+  L.hq = take(q ? RT * F * 2 : 0);
+  L.hexp = take(q ? RT * 4 : 0);
+  L.y = take(R * D * 2);
+  L.ysh = take(S * T * D * 2);
+  L.total = o;
+  return L;
+}
+
+moe_status check_desc(const moe_layer_desc* d) {
+  if (!d) return MOE_ERR_INVALID_ARG;
+  if (d->T < 0 || d->d_model <= 0 || d->d_ff <= 0 || d->n_experts <= 0 || d->top_k <= 0 || d->n_shared < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (d->wdtype < MOE_W_BF16 || d->wdtype > MOE_W_INT4_G128) return MOE_ERR_INVALID_ARG;
+  if (d->router_fp32 != 0 && d->router_fp32 != 1) return MOE_ERR_INVALID_ARG;
+  const int blk = d->wdtype == MOE_W_INT4_G128 ? 128 : 32;
+  if (d->d_model % blk || d->d_ff % blk) return MOE_ERR_INVALID_ARG;
+  if (d->top_k > d->n_experts || d->top_k > 32) return MOE_ERR_INVALID_ARG;
+  if (d->n_experts > 1024 || d->n_shared > 64) return MOE_ERR_UNSUPPORTED;
+  const int64_t rows = (int64_t)d->T * d->top_k + (int64_t)d->n_shared * d->T;
+  if (rows * (int64_t)(d->d_ff > d->d_model ? d->d_ff : d->d_model) > (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+struct DevInfo {
+  int sms = 0, smem_optin = 0;
+};
+
+DevInfo dev_info() {
+  static std::mutex mu;
+  static DevInfo cache[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  std::lock_guard<std::mutex> lk(mu);
+  if (cache[dev].sms == 0) {
+    cudaDeviceGetAttribute(&cache[dev].sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&cache[dev].smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  }
+  return cache[dev];
+}
+
+moe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// Fill the stream-kernel arguments of one stage.
+moe_status check_weights(const moe_layer_desc& d, const moe_weights* w, int n_expected) {
+  if (!w || !w->w13 || !w->w2) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w->w13) || !aligned16(w->w2)) return MOE_ERR_INVALID_ARG;
+  if (is4bit(d.wdtype)) {
+    if (!w->s13 || !w->s2 || !aligned16(w->s13) || !aligned16(w->s2)) return MOE_ERR_INVALID_ARG;
+  }
+  if (d.wdtype == MOE_W_NVFP4 && (!w->g13 || !w->g2)) return MOE_ERR_INVALID_ARG;
+  if ((w->stride_w13 | w->stride_s13 | w->stride_w2 | w->stride_s2) & 15) return MOE_ERR_INVALID_ARG;
+  if (w->stride_w13 < 0 || w->stride_s13 < 0 || w->stride_w2 < 0 || w->stride_s2 < 0) return MOE_ERR_INVALID_ARG;
+  if (w->n_physical < 0) return MOE_ERR_INVALID_ARG;
+  (void)n_expected;
+  return MOE_OK;
+}
+
+moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, const moe_weights* shared,
+                            const int32_t* offsets, const int32_t* row_token, const void* x, void* y_perm,
+                            void* y_shared, uint8_t* ws, cudaStream_t st) {
+  const Layout L = layout_of(d);
+  const int f = d.wdtype;
+  const bool q = is4bit(f);
+  const int T = d.T, D = d.d_model, F = d.d_ff, S = d.n_shared, E = d.n_experts, k = d.top_k;
+  const int R = T * k, RT = R + S * T;
+  const DevInfo di = dev_info();
+  cudaError_t err;
+  __half* xq = reinterpret_cast<__half*>(ws + L.xq);
+  int32_t* xexp = reinterpret_cast<int32_t*>(ws + L.xexp);
+  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
+  __half* hq = reinterpret_cast<__half*>(ws + L.hq);
+  int32_t* hexp = reinterpret_cast<int32_t*>(ws + L.hexp);
+  if (q) {
+    err = launch_prep_rows(x, T, D, f == MOE_W_INT4_G128, xq, xexp, st);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  auto fill = [&](FfnArgs& a, bool stage1) {
+    std::memset(&a, 0, sizeof(a));
+    const int64_t N = stage1 ? 2 * (int64_t)F : D, K = stage1 ? D : F;
+    const void* wv = stage1 ? routed->w13 : routed->w2;
+    const void* sv = stage1 ? routed->s13 : routed->s2;
+    int64_t sw = stage1 ? routed->stride_w13 : routed->stride_w2;
+    int64_t ss = stage1 ? routed->stride_s13 : routed->stride_s2;
+    a.w = static_cast<const uint8_t*>(wv);
+    a.s = static_cast<const uint8_t*>(sv);
+    a.gsc = stage1 ? routed->g13 : routed->g2;
+    a.stride_w = sw ? sw : mat_bytes(f, N, K);
+    a.stride_s = ss ? ss : scale_bytes(f, N, K);
+    a.slot_map = routed->slot_map;
+    a.n_phys = routed->n_physical ? routed->n_physical : E;
+    if (S > 0) {
+      a.w_sh = static_cast<const uint8_t*>(stage1 ? shared->w13 : shared->w2);
+      a.s_sh = static_cast<const uint8_t*>(stage1 ? shared->s13 : shared->s2);
+      a.gsc_sh = stage1 ? shared->g13 : shared->g2;
+      const int64_t shw = stage1 ? shared->stride_w13 : shared->stride_w2;
+      const int64_t shs = stage1 ? shared->stride_s13 : shared->stride_s2;
+      a.stride_w_sh = shw ? shw : mat_bytes(f, N, K);
+      a.stride_s_sh = shs ? shs : scale_bytes(f, N, K);
+    }
+    a.n_shared = S;
+    a.E = E;
+    a.T = T;
+    a.k = k;
+    a.N = stage1 ? F : D;
+    a.K = (int)K;
+    a.offsets = offsets;
+    a.row_token = row_token;
+  };
+  FfnArgs a1;
+  fill(a1, true);
+  a1.xsrc = static_cast<const uint8_t*>(q ? static_cast<const void*>(xq) : x);
+  a1.xexp = q ? xexp : nullptr;
+  a1.out_routed = h;
+  a1.out_shared = nullptr;
+  int unsup = 0;
+  err = launch_ffn_stream(f, true, a1, T, di.sms, di.smem_optin, st, &unsup);
+  if (unsup) return MOE_ERR_UNSUPPORTED;
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  if (q) {
+    err = launch_prep_rows(h, RT, F, f == MOE_W_INT4_G128, hq, hexp, st);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  FfnArgs a2;
+  fill(a2, false);
+  a2.xsrc = reinterpret_cast<const uint8_t*>(q ? static_cast<void*>(hq) : static_cast<void*>(h));
+  a2.xexp = q ? hexp : nullptr;
+  a2.out_routed = static_cast<__nv_bfloat16*>(y_perm);
+  a2.out_shared = static_cast<__nv_bfloat16*>(y_shared);
+  err = launch_ffn_stream(f, false, a2, T, di.sms, di.smem_optin, st, &unsup);
+  if (unsup) return MOE_ERR_UNSUPPORTED;
+  return from_cuda(err);
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_workspace_size(const moe_layer_desc* desc, size_t* bytes) {
+  moe_status s = check_desc(desc);
+  if (s != MOE_OK) return s;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = layout_of(*desc).total;
+  return MOE_OK;
+}
+
+moe_status moe_workspace_layout_of(const moe_layer_desc* desc, moe_workspace_layout* out) {
+  moe_status s = check_desc(desc);
+  if (s != MOE_OK) return s;
+  if (!out) return MOE_ERR_INVALID_ARG;
+  const Layout L = layout_of(*desc);
+  out->topk_idx = L.topk_idx;
+  out->topk_w = L.topk_w;
+  out->offsets = L.offsets;
+  out->row_token = L.row_token;
+  out->inv = L.inv;
+  out->total = L.total;
+  return MOE_OK;
+}
+
+moe_status moe_route_topk(const moe_layer_desc* desc, const void* x, const void* w_router, const float* logit_bias,
+                          int32_t* topk_idx, float* topk_w, void* workspace, size_t ws_bytes, void* stream) {
+  moe_status s = check_desc(desc);
+  if (s != MOE_OK) return s;
+  if (desc->T == 0) return MOE_OK;
+  if (!x || !w_router || !topk_idx || !topk_w || !workspace) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(workspace)) return MOE_ERR_INVALID_ARG;
+  const Layout L = layout_of(*desc);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  float* logits = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + L.logits);
+  return from_cuda(launch_route_topk(*desc, x, w_router, logit_bias, logits, topk_idx, topk_w,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_permute(const moe_layer_desc* desc, const int32_t* topk_idx, int32_t* offsets, int32_t* row_token,
+                       int32_t* inv, void* stream) {
+  moe_status s = check_desc(desc);
+  if (s != MOE_OK) return s;
+  if (!offsets) return MOE_ERR_INVALID_ARG;
+  if (desc->T > 0 && (!topk_idx || !row_token || !inv)) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_permute(topk_idx, desc->T, desc->top_k, desc->n_experts, offsets, row_token, inv,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_grouped_ffn(const moe_layer_desc* desc, const moe_weights* routed, const moe_weights* shared,
+                           const int32_t* offsets, const int32_t* row_token, const void* x, void* y_perm,
+                           void* y_shared, void* workspace, size_t ws_bytes, void* stream) {
+  moe_status s = check_desc(desc);
+  if (s != MOE_OK) return s;
+  if (desc->T == 0) return MOE_OK;
+  if ((s = check_weights(*desc, routed, desc->n_experts)) != MOE_OK) return s;
+  if (desc->n_shared > 0) {
+    if ((s = check_weights(*desc, shared, desc->n_shared)) != MOE_OK) return s;
+    if (!y_shared || !aligned16(y_shared)) return MOE_ERR_INVALID_ARG;
+  }
+  if (!offsets || !row_token || !x || !y_perm || !workspace) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y_perm) || !aligned16(workspace)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < layout_of(*desc).total) return MOE_ERR_WORKSPACE;
+  return grouped_ffn_impl(*desc, routed, shared, offsets, row_token, x, y_perm, y_shared,
+                          static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_combine(const moe_layer_desc* desc, const void* y_perm, const int32_t* inv, const float* topk_w,
+                       const void* y_shared, void* out, void* stream) {
+  moe_status s = check_desc(desc);
+  if (s != MOE_OK) return s;
+  if (desc->T == 0) return MOE_OK;
+  if (!y_perm || !inv || !topk_w || !out) return MOE_ERR_INVALID_ARG;
+  if (desc->n_shared > 0 && !y_shared) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_perm) || !aligned16(out) || (y_shared && !aligned16(y_shared))) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_combine(y_perm, inv, topk_w, y_shared, desc->n_shared, desc->T, desc->d_model,
+                                  desc->top_k, out, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_layer_forward(const moe_layer_desc* desc, const void* x, const void* w_router,
+                             const float* logit_bias, const moe_weights* routed, const moe_weights* shared,
+                             void* out, void* workspace, size_t ws_bytes, void* stream) {
+  moe_status s = check_desc(desc);
+  if (s != MOE_OK) return s;
+  if (desc->T == 0) return MOE_OK;
+  if ((s = check_weights(*desc, routed, desc->n_experts)) != MOE_OK) return s;
+  if (desc->n_shared > 0 && (s = check_weights(*desc, shared, desc->n_shared)) != MOE_OK) return s;
+  if (!x || !w_router || !out || !workspace) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(out) || !aligned16(workspace)) return MOE_ERR_INVALID_ARG;
+  const Layout L = layout_of(*desc);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + L.topk_idx);
+  float* gw = reinterpret_cast<float*>(ws + L.topk_w);
+  int32_t* offs = reinterpret_cast<int32_t*>(ws + L.offsets);
+  int32_t* rtok = reinterpret_cast<int32_t*>(ws + L.row_token);
+  int32_t* inv = reinterpret_cast<int32_t*>(ws + L.inv);
+  cudaError_t err = launch_route_topk(*desc, x, w_router, logit_bias, reinterpret_cast<float*>(ws + L.logits), idx,
+                                      gw, st);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  err = launch_permute(idx, desc->T, desc->top_k, desc->n_experts, offs, rtok, inv, st);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  void* y = ws + L.y;
+  void* ysh = desc->n_shared ? ws + L.ysh : nullptr;
+  s = grouped_ffn_impl(*desc, routed, shared, offs, rtok, x, y, ysh, ws, st);
+  if (s != MOE_OK) return s;
+  return from_cuda(launch_combine(y, inv, gw, ysh, desc->n_shared, desc->T, desc->d_model, desc->top_k, out, st));
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_OOM: return "out of memory";
+    case MOE_ERR_CACHE_PINNED_FULL: return "every cache slot of the layer is protected";
+    case MOE_ERR_TIMEOUT: return "a device-side wait timed out";
+    case MOE_ERR_INJECTED: return "injected fault";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_DEVICE_INDEX: return "a kernel saw an index out of range";
+  }
+  return "unknown status";
+}
+
+moe_status moe_get_last_error(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, moe::g_status, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(moe::g_status, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  return static_cast<moe_status>(v);
+}
+
+}  // extern "C"

@@ -1,0 +1,241 @@
+// Token permutation into per-expert groups, activation preparation, and the
+// weighted combine back to token order.
+//
+// Grouping: tokens that select the same expert are grouped so that one read of
+// the expert's weights serves all of them ("Understanding MoE Inference Costs
+// on Galactus", section "Prompt processing is a different phase").  The
+// grouping is a stable counting sort of the T*k (token, slot) pairs by expert:
+// per-expert counts, their exclusive prefix sum (offsets), then each pair's
+// row = offsets[e] + (number of earlier pairs with the same expert).  One
+// 1024-thread block does it: shared-memory histogram, block scan, then warp w
+// scans the pairs for experts w, w+32, ... with warp ballots, so the result
+// is independent of thread scheduling.
+//
+// Combine: out[t] = sum_j g[t,j] * y[inv[t*k+j]] + sum_s y_shared[s][t], fp32
+// in that order ("Each token is sent to the shared expert and also to one of
+// the 128 routed experts": "Mixture of experts VRAM: total vs active
+// parameters", section "How current MoE models route each token").
+#include "common.cuh"
+#include "profile.cuh"
+
+namespace moe {
+
+constexpr int kPermThreads = 1024;
+constexpr int kPermTile = 8192;
+
+__global__ void __launch_bounds__(kPermThreads)
+    permute_kernel(const int32_t* __restrict__ idx, int n, int k, int E, int32_t* __restrict__ offsets,
+                   int32_t* __restrict__ row_token, int32_t* __restrict__ inv) {
+  extern __shared__ int sm[];
+  int* counts = sm;            // [E]
+  int* cursor = sm + E;        // [E]
+  int* tile = sm + 2 * E;      // [kPermTile]
+  __shared__ int wsum[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int e = tid; e < E; e += kPermThreads) counts[e] = 0;
+  __syncthreads();
+  for (int i = tid; i < n; i += kPermThreads) {
+    const int e = __ldg(idx + i);
+    if (e < 0 || e >= E) {
+      set_status(MOE_ERR_DEVICE_INDEX);
+      inv[i] = -1;
+    } else {
+      atomicAdd(&counts[e], 1);
+    }
+  }
+  __syncthreads();
+  // exclusive scan over E <= 1024 counts (one per thread)
+  const int v = tid < E ? counts[tid] : 0;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = wsum[lane];
+    int wi = w;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, wi, off);
+      if (lane >= off) wi += o;
+    }
+    wsum[lane] = wi - w;  // exclusive prefix of warp totals
+  }
+  __syncthreads();
+  const int excl = incl - v + wsum[warp];
+  if (tid < E) {
+    cursor[tid] = excl;
+    offsets[tid] = excl;
+    if (tid == E - 1) offsets[E] = excl + v;
+  }
+  __syncthreads();
+  for (int base = 0; base < n; base += kPermTile) {
+    const int tn = min(kPermTile, n - base);
+    for (int i = tid; i < tn; i += kPermThreads) tile[i] = __ldg(idx + base + i);
+    __syncthreads();
+    for (int e = warp; e < E; e += kPermThreads / 32) {
+      int run = cursor[e];
+      for (int c0 = 0; c0 < tn; c0 += 32) {
+        const int i = c0 + lane;
+        const bool hit = i < tn && tile[i] == e;
+        const uint32_t m = __ballot_sync(0xffffffffu, hit);
+        if (hit) {
+          const int r = run + __popc(m & ((1u << lane) - 1u));
+          row_token[r] = (base + i) / k;
+          inv[base + i] = r;
+        }
+        run += __popc(m);
+      }
+      if (lane == 0) cursor[e] = run;
+    }
+    __syncthreads();
+  }
+}
+
+cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* offsets, int32_t* row_token,
+                           int32_t* inv, cudaStream_t st) {
+  const size_t smem = (size_t)(2 * E + kPermTile) * sizeof(int);
+  cudaError_t err = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  ProfScope prof("permute", st);
+  permute_kernel<<<1, kPermThreads, smem, st>>>(idx, T * k, k, E, offsets, row_token, inv);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Activation rows -> fp16 for the 4-bit weight paths.  Each row is scaled by
+// 2^-p with p = floor(log2(max|row|)) - 14 so that its largest magnitude lies
+// in [2^14, 2^15) (fp16's range); rexp[row] = p is undone on the accumulators.
+// With kPermInt4 each 8-element group is stored in the order
+// 0,4,1,5,2,6,3,7, the pairing the INT4 decoder produces.
+constexpr int kPrepThreads = 128;
+
+template <bool kPermInt4>
+__global__ void __launch_bounds__(kPrepThreads)
+    prep_rows_kernel(const __nv_bfloat16* __restrict__ src, int K, __half* __restrict__ dst,
+                     int32_t* __restrict__ rexp) {
+  const int row = blockIdx.x;
+  const int tid = threadIdx.x;
+  const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)row * K);
+  const int nchunk = K / 8;
+  float amax = 0.f;
+  for (int c = tid; c < nchunk; c += kPrepThreads) {
+    const uint4 u = __ldg(s + c);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      amax = fmaxf(amax, fabsf(bf16_bits_to_f32(w[q] & 0xffffu)));
+      amax = fmaxf(amax, fabsf(bf16_bits_to_f32(w[q] >> 16)));
+    }
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  __shared__ float red[kPrepThreads / 32];
+  if ((tid & 31) == 0) red[tid >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int w = 1; w < kPrepThreads / 32; ++w) amax = fmaxf(amax, red[w]);
+  int p = 0;
+  if (amax > 0.f && amax <= 3.0e38f) {
+    int ex;
+    frexpf(amax, &ex);  // amax = m * 2^ex, m in [0.5, 1)
+    p = ex - 15;        // floor(log2(amax)) - 14
+  }
+  if (tid == 0) rexp[row] = p;
+  const float scale = ldexpf(1.f, -p);
+  uint4* d = reinterpret_cast<uint4*>(dst + (size_t)row * K);
+  for (int c = tid; c < nchunk; c += kPrepThreads) {
+    const uint4 u = __ldg(s + c);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    float f[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      f[2 * q] = bf16_bits_to_f32(w[q] & 0xffffu) * scale;
+      f[2 * q + 1] = bf16_bits_to_f32(w[q] >> 16) * scale;
+    }
+    __half h[8];
+    if (kPermInt4) {
+      const int order[8] = {0, 4, 1, 5, 2, 6, 3, 7};
+#pragma unroll
+      for (int q = 0; q < 8; ++q) h[q] = __float2half_rn(f[order[q]]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) h[q] = __float2half_rn(f[q]);
+    }
+    d[c] = *reinterpret_cast<uint4*>(h);
+  }
+}
+
+cudaError_t launch_prep_rows(const void* src, int rows, int K, bool perm_int4, void* dst, int32_t* rexp,
+                             cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  ProfScope prof("prep_rows", st);
+  if (perm_int4)
+    prep_rows_kernel<true><<<rows, kPrepThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(src), K,
+                                                          static_cast<__half*>(dst), rexp);
+  else
+    prep_rows_kernel<false><<<rows, kPrepThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(src), K,
+                                                           static_cast<__half*>(dst), rexp);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+constexpr int kCombineThreads = 128;
+
+__global__ void __launch_bounds__(kCombineThreads)
+    combine_kernel(const __nv_bfloat16* __restrict__ y, const int32_t* __restrict__ inv,
+                   const float* __restrict__ gw, const __nv_bfloat16* __restrict__ y_shared, int n_shared, int T,
+                   int d, int k, __nv_bfloat16* __restrict__ out) {
+  const int t = blockIdx.x;
+  const int nchunk = d / 8;
+  const int nrows = T * k;
+  for (int c = threadIdx.x; c < nchunk; c += kCombineThreads) {
+    float acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int r = __ldg(inv + (size_t)t * k + j);
+      if (r < 0 || r >= nrows) {
+        set_status(MOE_ERR_DEVICE_INDEX);
+        continue;
+      }
+      const float g = __ldg(gw + (size_t)t * k + j);
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(y + (size_t)r * d) + c);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc[2 * q] = fmaf(g, bf16_bits_to_f32(w[q] & 0xffffu), acc[2 * q]);
+        acc[2 * q + 1] = fmaf(g, bf16_bits_to_f32(w[q] >> 16), acc[2 * q + 1]);
+      }
+    }
+    for (int s = 0; s < n_shared; ++s) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(y_shared + ((size_t)s * T + t) * d) + c);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc[2 * q] += bf16_bits_to_f32(w[q] & 0xffffu);
+        acc[2 * q + 1] += bf16_bits_to_f32(w[q] >> 16);
+      }
+    }
+    __nv_bfloat16 o[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) o[q] = __float2bfloat16_rn(acc[q]);
+    reinterpret_cast<uint4*>(out + (size_t)t * d)[c] = *reinterpret_cast<uint4*>(o);
+  }
+}
+
+cudaError_t launch_combine(const void* y, const int32_t* inv, const float* gw, const void* y_shared, int n_shared,
+                           int T, int d, int k, void* out, cudaStream_t st) {
+  if (T <= 0) return cudaSuccess;
+  ProfScope prof("combine", st);
+  combine_kernel<<<T, kCombineThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(y), inv, gw,
+                                                static_cast<const __nv_bfloat16*>(y_shared), n_shared, T, d, k,
+                                                static_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,184 @@
+// Router product and top-k selection with renormalised softmax gates.
+//
+// The router is the dense per-token scoring that "picks a few" experts
+// ("Mixture of experts VRAM: total vs active parameters", section "How current
+// MoE models route each token"); every token goes to a fixed number k of
+// experts (same section).  Selection is on the logits (softmax is monotone),
+// largest first, the lower expert index winning ties; the gates are the
+// softmax of the selected logits, which equals the softmax over all E experts
+// renormalised over the selection.
+//
+// Kernel 1 (router_logits_kernel): a block computes an 8-token x 4-expert tile
+// of logits.  Thread t of 256 owns the 8-element chunks t, t+256, ... of the
+// hidden dimension, accumulates its products in fp32 in that order, then the
+// partial sums are folded by a warp butterfly and the 8 warps are added in a
+// fixed order.  Every logit - every expert column - goes through the same
+// summation tree (depth MOE_ROUTER_SUM_DEPTH(d)), so identical router rows
+// give bit-identical logits and ties resolve exactly.
+//
+// Kernel 2 (topk_kernel): one warp per token.  k rounds of a warp-wide
+// argmax over (logit desc, index asc); gates from expf in fp32.
+#include "common.cuh"
+#include "profile.cuh"
+
+namespace moe {
+
+constexpr int kRouterTokens = 8;   // tokens per block
+constexpr int kRouterExperts = 4;  // experts per block
+constexpr int kRouterThreads = 256;
+
+template <bool kFp32Router>
+__global__ void __launch_bounds__(kRouterThreads)
+    router_logits_kernel(const __nv_bfloat16* __restrict__ x, const void* __restrict__ wr,
+                         const float* __restrict__ bias, float* __restrict__ logits, int T, int d, int E) {
+  const int t0 = blockIdx.x * kRouterTokens;
+  const int e0 = blockIdx.y * kRouterExperts;
+  const int tid = threadIdx.x;
+  const int nt = min(kRouterTokens, T - t0);
+  const int ne = min(kRouterExperts, E - e0);
+  float acc[kRouterTokens][kRouterExperts];
+#pragma unroll
+  for (int a = 0; a < kRouterTokens; ++a)
+#pragma unroll
+    for (int b = 0; b < kRouterExperts; ++b) acc[a][b] = 0.f;
+
+  const int nchunk = d / 8;
+  for (int c = tid; c < nchunk; c += kRouterThreads) {
+    float wv[kRouterExperts][8];
+#pragma unroll
+    for (int b = 0; b < kRouterExperts; ++b) {
+      const int e = e0 + (b < ne ? b : 0);
+      if constexpr (kFp32Router) {
+        const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(wr) + (size_t)e * d + c * 8);
+        float4 u0 = __ldg(p), u1 = __ldg(p + 1);
+        wv[b][0] = u0.x; wv[b][1] = u0.y; wv[b][2] = u0.z; wv[b][3] = u0.w;
+        wv[b][4] = u1.x; wv[b][5] = u1.y; wv[b][6] = u1.z; wv[b][7] = u1.w;
+      } else {
+        uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(wr) + (size_t)e * d + c * 8));
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          wv[b][2 * q] = bf16_bits_to_f32(w4[q] & 0xffffu);
+          wv[b][2 * q + 1] = bf16_bits_to_f32(w4[q] >> 16);
+        }
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < kRouterTokens; ++a) {
+      const int t = t0 + (a < nt ? a : 0);
+      uint4 u = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d + c * 8));
+      const uint32_t x4[4] = {u.x, u.y, u.z, u.w};
+      float xv[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        xv[2 * q] = bf16_bits_to_f32(x4[q] & 0xffffu);
+        xv[2 * q + 1] = bf16_bits_to_f32(x4[q] >> 16);
+      }
+#pragma unroll
+      for (int b = 0; b < kRouterExperts; ++b)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[a][b] = __fadd_rn(acc[a][b], __fmul_rn(xv[q], wv[b][q]));
+    }
+  }
+  // warp butterfly (identical association in every lane and every column)
+#pragma unroll
+  for (int a = 0; a < kRouterTokens; ++a)
+#pragma unroll
+    for (int b = 0; b < kRouterExperts; ++b)
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) acc[a][b] = __fadd_rn(acc[a][b], __shfl_xor_sync(0xffffffffu, acc[a][b], off));
+
+  __shared__ float part[kRouterThreads / 32][kRouterTokens * kRouterExperts];
+  const int warp = tid >> 5, lane = tid & 31;
+  if (lane == 0) {
+#pragma unroll
+    for (int a = 0; a < kRouterTokens; ++a)
+#pragma unroll
+      for (int b = 0; b < kRouterExperts; ++b) part[warp][a * kRouterExperts + b] = acc[a][b];
+  }
+  __syncthreads();
+  if (tid < kRouterTokens * kRouterExperts) {
+    const int a = tid / kRouterExperts, b = tid % kRouterExperts;
+    float s = part[0][tid];
+#pragma unroll
+    for (int w = 1; w < kRouterThreads / 32; ++w) s = __fadd_rn(s, part[w][tid]);
+    if (a < nt && b < ne) {
+      const int e = e0 + b;
+      if (bias != nullptr) s = __fadd_rn(s, __ldg(bias + e));
+      logits[(size_t)(t0 + a) * E + e] = s;
+    }
+  }
+}
+
+// (value, index) ordering: larger value first, then lower index.  NaN never wins.
+__device__ __forceinline__ bool beats(float v, int i, float w, int j) {
+  return (v > w) || (v == w && i < j);
+}
+
+__global__ void __launch_bounds__(256)
+    topk_kernel(const float* __restrict__ logits, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                int T, int E, int k) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= T) return;
+  const float* lt = logits + (size_t)warp * E;
+  int prev_i = -1;
+  float prev_v = __int_as_float(0x7f800000);  // +inf: everything is below the previous pick
+  float my_v = 0.f;
+  int my_i = -1;
+  for (int j = 0; j < k; ++j) {
+    // best element strictly after (prev_v, prev_i) in the total order
+    float bv = __int_as_float(0xff800000);  // -inf
+    int bi = 0x7fffffff;
+    for (int e = lane; e < E; e += 32) {
+      const float v = lt[e];
+      if (v != v) continue;  // NaN is never selected
+      if (!beats(prev_v, prev_i, v, e)) continue;
+      if (beats(v, e, bv, bi)) { bv = v; bi = e; }
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (beats(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+    }
+    if (bi == 0x7fffffff || bi < 0 || bi >= E) {
+      bi = -1;
+      if (lane == 0) set_status(MOE_ERR_DEVICE_INDEX);
+    }
+    if (lane == j) { my_v = bv; my_i = bi; }
+    prev_v = bv;
+    prev_i = bi;
+  }
+  // gates: softmax over the selected logits (lane j holds pick j; pick 0 is the max)
+  const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
+  const float ex = (lane < k) ? expf(my_v - vmax) : 0.f;
+  float sum = 0.f;
+  for (int j = 0; j < k; ++j) sum = __fadd_rn(sum, __shfl_sync(0xffffffffu, ex, j));
+  if (lane < k) {
+    topk_idx[(size_t)warp * k + lane] = my_i;
+    topk_w[(size_t)warp * k + lane] = ex / sum;
+  }
+}
+
+cudaError_t launch_route_topk(const moe_layer_desc& dsc, const void* x, const void* wr, const float* bias,
+                              float* logits, int32_t* topk_idx, float* topk_w, cudaStream_t st) {
+  const int T = dsc.T, d = dsc.d_model, E = dsc.n_experts, k = dsc.top_k;
+  dim3 grid(ceil_div(T, kRouterTokens), ceil_div(E, kRouterExperts));
+  {
+  ProfScope prof("router_logits", st);
+  if (dsc.router_fp32)
+    router_logits_kernel<true><<<grid, kRouterThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x), wr, bias,
+                                                                  logits, T, d, E);
+  else
+    router_logits_kernel<false><<<grid, kRouterThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x), wr, bias,
+                                                                   logits, T, d, E);
+  }
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  ProfScope prof("topk", st);
+  topk_kernel<<<ceil_div(T * 32, 256), 256, 0, st>>>(logits, topk_idx, topk_w, T, E, k);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -195,17 +195,25 @@ def encode_matrix(w: torch.Tensor, wdtype: str) -> Dict[str, torch.Tensor]:
 # Layer draws
 # ----------------------------------------------------------------------------
 
-def draw_experts(shape: LayerShape, n: int, seed: int, device="cpu", chunk: int = 8):
+EXPERT_CHUNK = 8
+
+
+def draw_experts(shape: LayerShape, n: int, seed: int, device="cpu", chunks: Optional[list] = None):
     """Draw and encode ``n`` experts of ``shape`` (W13 and W2).
 
     Returns dict with keys w13, s13, g13, w2, s2, g2 (absent keys = not used by
-    the format).  Experts are drawn ``chunk`` at a time to bound memory.
+    the format).  Experts are drawn EXPERT_CHUNK at a time, each chunk from its
+    own generator seeded by (seed, chunk), so that a subset of chunks can be
+    drawn alone (``chunks``: list of chunk indices; the result then holds only
+    those chunks' experts, in order).
     """
     d, f = shape.d_model, shape.d_ff
-    gen = _gen(seed, device)
     parts13, parts2 = [], []
-    for e0 in range(0, n, chunk):
-        m = min(chunk, n - e0)
+    todo = range(0, (n + EXPERT_CHUNK - 1) // EXPERT_CHUNK) if chunks is None else chunks
+    for ci in todo:
+        e0 = ci * EXPERT_CHUNK
+        m = min(EXPERT_CHUNK, n - e0)
+        gen = _gen(seed * 65537 + ci, device)
         w13 = torch.randn(m, 2 * f, d, generator=gen, device=device) * shape.weight_std
         w2 = torch.randn(m, d, f, generator=gen, device=device) * shape.weight_std
         parts13.append(encode_matrix(w13, shape.wdtype))

@@ -95,8 +95,18 @@ def unpack_nibbles(packed) -> np.ndarray:
     return out
 
 
-def _expand_blocks(scale: np.ndarray, block: int) -> np.ndarray:
-    return np.repeat(scale, block, axis=-1)
+def _decode_codes(codes: np.ndarray, element_decoder) -> np.ndarray:
+    """Apply a 4-bit element decoder through its 16-entry table (same values,
+    one lookup per element)."""
+    table = element_decoder(np.arange(16))
+    return table[codes]
+
+
+def _times_blocks(values: np.ndarray, scale: np.ndarray, block: int) -> np.ndarray:
+    """values [..., K] * scale [..., K/block], each scale covering `block` consecutive K."""
+    shp = values.shape
+    v = values.reshape(shp[:-1] + (shp[-1] // block, block))
+    return (v * scale[..., None]).reshape(shp)
 
 
 def dequant(wdtype: str, w, s=None, g=None) -> np.ndarray:
@@ -110,15 +120,15 @@ def dequant(wdtype: str, w, s=None, g=None) -> np.ndarray:
         return bf16_bits_to_f64(w)
     codes = unpack_nibbles(w)
     if wdtype == "mxfp4":
-        return e2m1_to_f64(codes) * _expand_blocks(e8m0_to_f64(s), 32)
+        return _times_blocks(_decode_codes(codes, e2m1_to_f64), e8m0_to_f64(s), 32)
     if wdtype == "nvfp4":
         gs = np.asarray(_as_np(g), dtype=np.float64)
-        v = e2m1_to_f64(codes) * _expand_blocks(e4m3_to_f64(s), 16)
+        v = _times_blocks(_decode_codes(codes, e2m1_to_f64), e4m3_to_f64(s), 16)
         if gs.ndim == 0:
             return v * gs
         return v * gs.reshape(gs.shape + (1,) * (v.ndim - gs.ndim))
     if wdtype == "int4":
-        return int4_to_f64(codes) * _expand_blocks(bf16_bits_to_f64(s), 128)
+        return _times_blocks(_decode_codes(codes, int4_to_f64), bf16_bits_to_f64(s), 128)
     raise ValueError(wdtype)
 
 

@@ -1,0 +1,180 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle.
+
+Shapes span several row tiles and K chunks with ragged tails (d, d_ff = 2880
+leave 64-row and 64-column remainders), multiple activation passes (experts
+with more than 32 rows), shared experts, every weight format, empty and
+degenerate cases.  Full-size configurations are checked on sampled tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+import gpu_harness as H
+
+pytestmark = pytest.mark.gpu
+
+
+def _layer(shape, T, seed, device="cpu", **kw):
+    """(layer for the oracle, the same layer on the GPU).  Full-size layers are
+    drawn on the GPU; the oracle then reads the experts it needs from there."""
+    hl = mi.draw_layer(shape, T, seed, device=device, **kw)
+    return hl, H.to_device(hl)
+
+
+CASES = [
+    # name, shape, T
+    ("tiny", mi.TINY, 16),
+    ("mxfp4_gptoss_dims", mi.GPTOSS.replace(n_experts=16), 8),
+    ("mxfp4_gptoss_dims_T1", mi.GPTOSS.replace(n_experts=16), 1),
+    ("mxfp4_many_rows", mi.GPTOSS.replace(n_experts=4, top_k=2, d_model=576, d_ff=832), 150),
+    ("int4_shared", mi.KIMI.replace(d_model=896, d_ff=384, n_experts=48), 40),
+    ("int4_shared_T1", mi.KIMI.replace(d_model=896, d_ff=384, n_experts=48), 1),
+    ("nvfp4_zipf", mi.BANK.replace(d_model=1024, d_ff=384, n_experts=32), 16),
+    ("bf16_passes", mi.MIXTRAL.replace(d_model=512, d_ff=1024), 100),
+    ("bf16_router_fp32_odd", mi.TINY.replace(d_model=320, d_ff=96, n_experts=7, top_k=3), 33),
+]
+
+
+@pytest.mark.parametrize("name,shape,T", CASES, ids=[c[0] for c in CASES])
+@pytest.mark.parametrize("seed", [0, 1])
+def test_layer_matches_oracle(name, shape, T, seed):
+    hl, dl = _layer(shape, T, seed)
+    res = H.run_layer(dl)
+    rel, n_amb = H.full_check(hl, res)
+    print(f"{name} seed={seed}: rel err {rel:.2e}, ambiguous tokens {n_amb}")
+
+
+@pytest.mark.parametrize("seed", [2])
+def test_tiny_seed2(seed):
+    hl, dl = _layer(mi.TINY, 16, seed)
+    H.full_check(hl, H.run_layer(dl))
+
+
+def test_stepwise_entry_points_equal_layer_forward():
+    for shape, T in [(mi.KIMI.replace(d_model=896, d_ff=384, n_experts=48), 12),
+                     (mi.GPTOSS.replace(n_experts=16), 5), (mi.TINY, 16)]:
+        hl, dl = _layer(shape, T, 3)
+        a = H.run_layer(dl)
+        b = H.run_steps(dl)
+        for key in ("out", "idx", "gates", "offsets", "row_token", "inv"):
+            assert torch.equal(a[key], b[key]), key
+
+
+def test_deterministic_across_runs():
+    hl, dl = _layer(mi.GPTOSS.replace(n_experts=32), 24, 4)
+    a = H.run_layer(dl)["out"].clone()
+    for _ in range(3):
+        assert torch.equal(a, H.run_layer(dl)["out"])
+
+
+def test_empty_batch_is_noop():
+    hl, dl = _layer(mi.TINY, 0, 0)
+    res = H.run_layer(dl)
+    assert res["out"].shape == (0, 256)
+
+
+def test_single_expert_dense_mlp():
+    shape = mi.TINY.replace(n_experts=1, top_k=1, router_fp32=False)
+    hl, dl = _layer(shape, 9, 5)
+    H.full_check(hl, H.run_layer(dl))
+
+
+def test_k_equals_E_with_zero_router_is_uniform_average():
+    shape = mi.GPTOSS.replace(n_experts=4, top_k=4, d_model=256, d_ff=256)
+    hl, dl = _layer(shape, 6, 6)
+    hl["router"] = torch.zeros_like(hl["router"])
+    dl["router"] = hl["router"].cuda()
+    res = H.run_layer(dl)
+    assert torch.allclose(res["gates"], torch.full_like(res["gates"], 0.25), atol=0, rtol=0)
+    assert res["idx"].cpu().tolist() == [[0, 1, 2, 3]] * 6  # ties: lower index first
+    H.full_check(hl, res)
+
+
+def test_identical_router_rows_tie_to_lower_index():
+    shape = mi.GPTOSS.replace(n_experts=8, top_k=2, d_model=256, d_ff=256)
+    hl, dl = _layer(shape, 20, 7)
+    r = hl["router"].clone()
+    r[5] = r[2]  # experts 2 and 5 always tie exactly
+    r[6] = r[1]
+    hl["router"] = r
+    dl["router"] = r.cuda()
+    res = H.run_layer(dl)
+    idx = res["idx"].cpu().numpy()
+    assert not np.any((idx == 5).any(1) & ~(idx == 2).any(1))  # 5 only ever chosen together with 2
+    H.full_check(hl, res)
+
+
+def test_identical_experts_reduce_to_one_ffn():
+    shape = mi.BANK.replace(d_model=512, d_ff=256, n_experts=16)
+    hl, dl = _layer(shape, 11, 8, identical_experts=True)
+    H.full_check(hl, H.run_layer(dl))
+
+
+def test_out_of_range_expert_index_sets_status():
+    import expert_ffn_layer_route_b200 as moe
+    moe.moe_get_last_error()
+    shape = mi.TINY
+    desc = moe.make_desc(shape, 4)
+    idx = torch.tensor([[0, 1], [2, 99], [3, 4], [5, 6]], dtype=torch.int32, device="cuda")
+    offs = torch.empty(shape.n_experts + 1, dtype=torch.int32, device="cuda")
+    rtok = torch.empty(8, dtype=torch.int32, device="cuda")
+    inv = torch.empty(8, dtype=torch.int32, device="cuda")
+    moe.moe_permute(desc, idx, offs, rtok, inv)
+    assert moe.moe_get_last_error() == 9
+    assert inv.cpu().tolist()[3] == -1
+    assert offs.cpu().tolist()[-1] == 7
+    assert moe.moe_get_last_error() == 0  # cleared
+
+
+# ------------------------------------------------------------ full sizes ----
+
+@pytest.mark.parametrize("shape,T", [(mi.GPTOSS, 64), (mi.GPTOSS, 1), (mi.KIMI, 128), (mi.BANK, 16),
+                                     (mi.MIXTRAL, 4096)])
+def test_full_size_routing_exact(shape, T):
+    """Router + top-k + permutation at the measured sizes, every token."""
+    import expert_ffn_layer_route_b200 as moe
+    from oracle import layer as OL
+    gen_dev = "cuda"
+    x = mi.draw_tokens(T, shape.d_model, 11, gen_dev)
+    router = mi.draw_router(shape, 11, gen_dev)
+    bias = mi.zipf_offsets(shape.n_experts, shape.zipf_s, 11, gen_dev) if shape.zipf_s else None
+    desc = moe.make_desc(shape, T)
+    ws = torch.empty(moe.moe_workspace_size(desc), dtype=torch.uint8, device="cuda")
+    idx = torch.empty(T, shape.top_k, dtype=torch.int32, device="cuda")
+    gw = torch.empty(T, shape.top_k, dtype=torch.float32, device="cuda")
+    moe.moe_route_topk(desc, x, router, bias, idx, gw, ws)
+    offs = torch.empty(shape.n_experts + 1, dtype=torch.int32, device="cuda")
+    rtok = torch.empty(T * shape.top_k, dtype=torch.int32, device="cuda")
+    inv = torch.empty(T * shape.top_k, dtype=torch.int32, device="cuda")
+    moe.moe_permute(desc, idx, offs, rtok, inv)
+    torch.cuda.synchronize()
+    hl = {"shape": shape, "x": x.cpu(), "router": router.cpu(), "bias": bias.cpu() if bias is not None else None}
+    xs, wr = OL.to_f64(hl["x"]), OL.to_f64(hl["router"])
+    b = OL.to_f64(hl["bias"]) if bias is not None else None
+    logits = OL.router_logits(xs, wr, b)
+    ridx, rg, margin = OL.topk_select(logits, shape.top_k)
+    beta = OL.logit_error_bound(xs, wr, b, moe.router_sum_depth(shape.d_model))
+    uniq = margin > 2 * beta
+    g_idx = idx.cpu().numpy()
+    assert np.array_equal(g_idx[uniq], ridx[uniq])
+    print(f"{shape.name} T={T}: ambiguous tokens {int((~uniq).sum())}")
+    c, o, rt, iv = OL.permute(g_idx, shape.n_experts)
+    assert np.array_equal(offs.cpu().numpy(), o)
+    assert np.array_equal(rtok.cpu().numpy(), rt)
+    assert np.array_equal(inv.cpu().numpy(), iv)
+    g = gw.cpu().double().numpy()
+    assert np.all(np.abs(g[uniq] - rg[uniq]) <= 1e-5 + 2 * rg[uniq] * beta[uniq, None])
+
+
+@pytest.mark.parametrize("shape,T,tokens", [(mi.GPTOSS, 64, [0, 13, 37, 63]), (mi.GPTOSS, 1, [0]),
+                                            (mi.KIMI, 128, [5, 77, 127]), (mi.BANK, 16, [0, 9, 15])])
+def test_full_size_layer_sampled_tokens(shape, T, tokens):
+    """Whole layer at the measured size (launch configuration of the benchmark);
+    the oracle recomputes a sample of tokens."""
+    hl, dl = _layer(shape, T, 12, device="cuda")
+    res = H.run_layer(dl)
+    ref, n_amb = H.check_routing(hl, res["idx"], res["gates"], tokens=tokens)
+    H.check_permutation(res, shape)
+    rel = H.check_output(res["out"], ref["out"], tokens=tokens)
+    print(f"{shape.name} T={T}: rel err {rel:.2e} on {len(tokens)} tokens, ambiguous {n_amb}")
