@@ -69,8 +69,8 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, bus_id: str):
-        self.bus_id = bus_id.lower()
+    def __init__(self, bus: int = -1):
+        self.bus = bus  # PCI bus number of the GPU under test (-1: take every row)
         self.proc = None
         self.lines = []
 
@@ -100,7 +100,11 @@ class ClockSampler:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 10:
                 continue
-            if self.bus_id and not parts[1].lower().endswith(self.bus_id[-12:]):
+            try:
+                bus = int(parts[1].split(":")[1], 16)
+            except (IndexError, ValueError):
+                bus = -1
+            if self.bus >= 0 and bus != self.bus:
                 continue
             rows.append(parts)
         if not rows:
@@ -286,9 +290,9 @@ def run_ours(args):
 
     moe.moe_profile_enable(True)
     moe.moe_profile_collect()
-    bus = ""
+    bus = -1
     try:
-        bus = torch.cuda.get_device_properties(dev).pci_bus_id
+        bus = int(torch.cuda.get_device_properties(dev).pci_bus_id)
     except Exception:
         pass
     clocks = ClockSampler(bus) if rank == 0 else None

@@ -14,17 +14,21 @@
 //   stage 1: h = silu(x W_gate^T) * (x W_up^T)   (gate and up tiles paired)
 //   stage 2: y = h W_down^T
 //
-// Block = 8 consumer warps + 1 producer warp.  The producer issues 1-D bulk
-// copies (cp.async.bulk, completion on mbarriers) of 128-byte row chunks of
-// the tile's weight rows and of the matching activation rows into a ring of
-// shared-memory stages; consumers decode the 4-bit codes to fp16 (E2M1 with
-// the hardware cvt, INT4 by the 1024-offset trick), and run m16n8k16 MMAs
-// with fp32 accumulation.  Block scales: MXFP4 (E8M0 per 32) and INT4 (bf16
-// per 128) multiply the fp32 partial sums of their block; NVFP4 (E4M3 per 16)
-// multiplies the fp16 weights (the product is exact in fp16) and its fp32
-// global scale is applied in the epilogue.  Within each 32-wide K block lane
-// c of a quad holds K = 8c..8c+7, i.e. the MMA's K order is a fixed
-// permutation of the block, applied identically to both operands.
+// Block = 8 consumer warps + 1 producer warp, one block per SM, persistent
+// over the work items.  The producer's elected lane issues TMA tiled loads
+// (128-row x 128-byte boxes, 128-byte swizzle) of the weights and of the
+// expert's activation rows into a ring of shared-memory stages, completing on
+// mbarriers.  Consumers decode the 4-bit codes to fp16 (E2M1 with the
+// hardware cvt, INT4 by the 1024-offset trick) and run m16n8k16 MMAs with
+// fp32 accumulation.  Block scales: MXFP4 (E8M0 per 32) and INT4 (bf16 per
+// 128) multiply the fp32 partial sums of their block; NVFP4 (E4M3 per 16)
+// multiplies the fp16 weights (exact in fp16) and its fp32 global scale is
+// applied in the epilogue.  Within each 32-wide K block lane c of a quad
+// holds K = 8c..8c+7, i.e. the MMA's K order is a fixed permutation of the
+// block, applied identically to both operands.  Activation rows (and bf16
+// weight rows) are read through the row order sigma(g) = (g>>1) | (g&1)<<2
+// inside each group of 8 so that the swizzled 16-byte reads are free of bank
+// conflicts; the epilogue maps columns (rows) back through the same sigma.
 #include "ffn_stream.cuh"
 #include "profile.cuh"
 
@@ -32,52 +36,48 @@ namespace moe {
 
 constexpr int kConsumerWarps = 8;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kRowsPerTile = 256;     // smem weight rows per item
-constexpr int kChunkBytes = 128;      // bytes of one weight row per stage
+constexpr int kRowsPerStage = 256;  // smem weight rows per stage (2 boxes of 128)
+constexpr int kBoxRows = 128;
+constexpr int kLine = 128;          // bytes per smem row (one swizzle line)
 constexpr int kMaxStages = 8;
 
 template <int F>
 struct FmtTraits;
 template <>
 struct FmtTraits<kBF16> {
-  static constexpr int kc = 64;       // K values per stage
-  static constexpr int sw = 192;      // smem weight row stride (bytes)
-  static constexpr int blk = 0;       // scale block (0: none)
-  static constexpr int sbytes = 0;    // bytes per scale
+  static constexpr int kc = 64;     // K values per stage (128 bytes of a weight row)
+  static constexpr int blk = 0;     // scale block (0: none)
+  static constexpr int sbytes = 0;  // bytes per scale
 };
 template <>
 struct FmtTraits<kMXFP4> {
-  static constexpr int kc = 256, sw = 144, blk = 32, sbytes = 1;
+  static constexpr int kc = 256, blk = 32, sbytes = 1;
 };
 template <>
 struct FmtTraits<kNVFP4> {
-  static constexpr int kc = 256, sw = 144, blk = 16, sbytes = 1;
+  static constexpr int kc = 256, blk = 16, sbytes = 1;
 };
 template <>
 struct FmtTraits<kINT4> {
-  static constexpr int kc = 256, sw = 144, blk = 128, sbytes = 2;
+  static constexpr int kc = 256, blk = 128, sbytes = 2;
 };
 
-template <int F>
-__device__ __forceinline__ int scale_row_bytes(int K) {
-  return FmtTraits<F>::blk ? (K / FmtTraits<F>::blk) * FmtTraits<F>::sbytes : 0;
-}
+__device__ __forceinline__ int sigma8(int g) { return (g >> 1) | ((g & 1) << 2); }
 
 // Everything a block needs to know about one work item.
 struct Item {
   int valid;
-  int shared_idx;   // >= 0 for a shared expert
-  int expert;       // logical expert (routed) or shared index
+  int shared_idx;  // >= 0 for a shared expert
   int tile;
-  int row_start;    // first routed row of the expert (routed), 0 for shared
-  int n_cols;       // rows of x this expert applies to
-  const uint8_t* wbase;
+  int xrow0;       // first activation / output row of this expert
+  int n_cols;      // activation rows of this expert
+  int phys;        // physical expert index (TMA coordinate)
   const uint8_t* sbase;
   float gscale;
 };
 
-template <int F, bool kGateUp>
-__device__ __forceinline__ Item decode_item(const FfnArgs& a, int item, int ntile, int n_act, const int* act,
+template <int F>
+__device__ __forceinline__ Item decode_item(const FfnArgs& a, int item, int ntile, const int* act,
                                             const int* offs) {
   Item it{};
   const int grp = item / ntile;
@@ -85,29 +85,26 @@ __device__ __forceinline__ Item decode_item(const FfnArgs& a, int item, int ntil
   it.valid = 1;
   if (grp < a.n_shared) {
     it.shared_idx = grp;
-    it.expert = grp;
-    it.row_start = 0;
+    it.xrow0 = a.T * a.k + grp * a.T;
     it.n_cols = a.T;
-    it.wbase = a.w_sh + (int64_t)grp * a.stride_w_sh;
+    it.phys = grp;
     it.sbase = a.s_sh ? a.s_sh + (int64_t)grp * a.stride_s_sh : nullptr;
     it.gscale = (F == kNVFP4 && a.gsc_sh) ? __ldg(a.gsc_sh + grp) : 1.f;
   } else {
     const int e = act[grp - a.n_shared];
     it.shared_idx = -1;
-    it.expert = e;
-    it.row_start = offs[e];
+    it.xrow0 = offs[e];
     it.n_cols = offs[e + 1] - offs[e];
     int p = a.slot_map ? __ldg(a.slot_map + e) : e;
     if (p == -1 && a.slot_map) {
       it.valid = 0;  // not resident in this call: skipped
       p = 0;
-    } else if (p < 0 || p >= a.n_phys || it.row_start < 0 || it.n_cols < 0 ||
-               it.row_start + it.n_cols > a.T * a.k) {
+    } else if (p < 0 || p >= a.n_phys || it.xrow0 < 0 || it.n_cols < 0 || it.xrow0 + it.n_cols > a.T * a.k) {
       set_status(MOE_ERR_DEVICE_INDEX);
       it.valid = 0;
       p = 0;
     }
-    it.wbase = a.w + (int64_t)p * a.stride_w;
+    it.phys = p;
     it.sbase = a.s ? a.s + (int64_t)p * a.stride_s : nullptr;
     it.gscale = (F == kNVFP4 && a.gsc) ? __ldg(a.gsc + e) : 1.f;
   }
@@ -115,17 +112,20 @@ __device__ __forceinline__ Item decode_item(const FfnArgs& a, int item, int ntil
 }
 
 template <int F, int NG, bool kGateUp>
-__global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const FfnArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const __grid_constant__ FfnArgs a) {
   using Tr = FmtTraits<F>;
   constexpr int KC = Tr::kc;
-  constexpr int SW = Tr::sw;
-  constexpr int SX = KC * 2 + 64;           // smem activation row stride (bytes)
-  constexpr int XCOLS = NG * 8;             // activation rows per pass
-  constexpr int kBlocksPerChunk = KC / 32;
+  constexpr int XCOLS = NG * 8;                 // activation rows per pass
+  constexpr int NXBOX = (KC * 2) / kLine;       // 128-byte activation boxes per stage
+  constexpr int W_BYTES = kRowsPerStage * kLine;
+  constexpr int X_BYTES = NXBOX * XCOLS * kLine;
+  constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
 
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment for the swizzled TMA destinations
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + kMaxStages;
   uint64_t* sfull = empty + kMaxStages;
@@ -133,14 +133,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const FfnArgs a
   volatile int* s_abort = reinterpret_cast<volatile int*>(sempty + 2);
   int* s_nact = reinterpret_cast<int*>(sempty + 2) + 1;
   int* s_offs = reinterpret_cast<int*>(sempty + 2) + 4;  // [E+1]
-  int* s_act = s_offs + (a.E + 4);           // [E]
-  uint8_t* s_scale = smem + (((16 * kMaxStages + 32 + 16 + 8 * a.E + 64) + 127) & ~127);
+  int* s_act = s_offs + (a.E + 4);                       // [E]
+  const int hdr = ((16 * kMaxStages + 32 + 16 + 8 * a.E + 64) + 1023) & ~1023;
+  uint8_t* s_scale = smem + hdr;
   uint8_t* s_stage = s_scale + a.n_scale_buf * a.smem_scale_bytes;
-  const int stage_w_bytes = kRowsPerTile * SW;
-  const int stage_bytes = stage_w_bytes + XCOLS * SX;
 
   const int E = a.E;
-  // ---- block setup: barriers, routed-expert list
   if (tid == 0) {
     for (int i = 0; i < a.n_stages; ++i) {
       mbar_init(&full[i], 1);
@@ -169,38 +167,45 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const FfnArgs a
   __syncthreads();
   const int n_act = *s_nact;
 
-  const int rows_per_item = kGateUp ? kRowsPerTile / 2 : kRowsPerTile;
+  const int rows_per_item = kGateUp ? kRowsPerStage / 2 : kRowsPerStage;
   const int ntile = ceil_div(a.N, rows_per_item);
   const int n_items = (a.n_shared + n_act) * ntile;
   const int K = a.K;
-  const int row_bytes = (F == kBF16) ? K * 2 : K / 2;  // weight row bytes
-  const int srow = scale_row_bytes<F>(K);
+  const int srow = Tr::blk ? (K / Tr::blk) * Tr::sbytes : 0;
   const int nchunks = ceil_div(K, KC);
   const int nstage = a.n_stages;
   const int nsb = a.n_scale_buf;
+  const int x_row_bytes = K * 2;
 
   if (warp == kConsumerWarps) {
     // ===================================================== producer warp
-    const uint64_t pol = l2_evict_first_policy();
-    uint32_t cnt = 0;  // stages issued
-    int item_no = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++item_no) {
-      const Item it = decode_item<F, kGateUp>(a, item, ntile, n_act, s_act, s_offs);
-      const int r0 = it.tile * rows_per_item;
-      const int nrows = min(rows_per_item, a.N - r0);  // valid rows per half
-      const int passes = it.valid ? ceil_div(it.n_cols, XCOLS) : 0;
-      const int sb = item_no % nsb;
-      const uint32_t suse = item_no / nsb;
-      const int sc_at = (nsb == 2) ? 0 : min(nstage - 1, nchunks - 1);
-      for (int pass = 0; pass < max(passes, 1); ++pass) {
-        const int c0 = pass * XCOLS;
-        const int ncols = passes ? min(XCOLS, it.n_cols - c0) : 0;
-        for (int ch = 0; ch < nchunks; ++ch) {
-          if (Tr::blk && pass == 0 && ch == sc_at) {
-            // block scales of the item's rows (whole K), one or two contiguous runs
-            if (!mbar_wait(&sempty[sb], (suse & 1u) ^ 1u)) { *s_abort = 1; }
-            if (*s_abort) break;
-            if (lane == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&a.tm_w);
+      prefetch_tmap(&a.tm_x);
+      if (a.n_shared) prefetch_tmap(&a.tm_wsh);
+      const uint64_t pol_w = l2_evict_first_policy();
+      const uint64_t pol_x = l2_evict_last_policy();
+      uint32_t cnt = 0;
+      int item_no = 0;
+      for (int item = blockIdx.x; item < n_items && !*s_abort; item += gridDim.x, ++item_no) {
+        const Item it = decode_item<F>(a, item, ntile, s_act, s_offs);
+        const int r0 = it.tile * rows_per_item;
+        const int nrows = min(rows_per_item, a.N - r0);
+        const int passes = it.valid ? ceil_div(it.n_cols, XCOLS) : 0;
+        const int sb = item_no % nsb;
+        const uint32_t suse = item_no / nsb;
+        const int sc_at = (nsb == 2) ? 0 : min(nstage - 1, nchunks - 1);
+        const CUtensorMap* tw = it.shared_idx >= 0 ? &a.tm_wsh : &a.tm_w;
+        // boxes of weight rows: stage 1 gate rows r0.. and up rows N+r0..; stage 2 rows r0.., r0+128..
+        const int nbox_w = kGateUp ? 2 : (nrows > kBoxRows ? 2 : 1);
+        for (int pass = 0; pass < max(passes, 1) && !*s_abort; ++pass) {
+          const int c0 = pass * XCOLS;
+          for (int ch = 0; ch < nchunks; ++ch) {
+            if (Tr::blk && pass == 0 && ch == sc_at) {
+              if (!mbar_wait(&sempty[sb], (suse & 1u) ^ 1u)) {
+                *s_abort = 1;
+                break;
+              }
               const uint32_t bytes = (uint32_t)(nrows * srow);
               mbar_arrive_expect_tx(&sfull[sb], it.valid ? bytes * (kGateUp ? 2u : 1u) : 0u);
               if (it.valid) {
@@ -210,49 +215,36 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const FfnArgs a
                   bulk_g2s(dst + rows_per_item * srow, it.sbase + (int64_t)(a.N + r0) * srow, bytes, &sfull[sb]);
               }
             }
-            __syncwarp();
-          }
-          const int s = cnt % nstage;
-          const uint32_t par = ((cnt / nstage) & 1u) ^ 1u;
-          if (!mbar_wait(&empty[s], par)) *s_abort = 1;
-          if (*s_abort) break;
-          const int kb = ch * kChunkBytes;  // byte offset of this chunk inside a weight row
-          const uint32_t wbytes = (uint32_t)min(kChunkBytes, row_bytes - kb);
-          const uint32_t xbytes = (uint32_t)(min(KC, K - ch * KC) * 2);
-          const int nw = it.valid ? (kGateUp ? 2 * nrows : nrows) : 0;
-          if (lane == 0) mbar_arrive_expect_tx(&full[s], nw * wbytes + ncols * xbytes);
-          __syncwarp();
-          uint8_t* sw_base = s_stage + s * stage_bytes;
-          for (int r = lane; r < nw; r += 32) {
-            int grow, srow_i;
-            if (kGateUp) {
-              const bool up = r >= nrows;
-              const int rr = up ? r - nrows : r;
-              grow = (up ? a.N : 0) + r0 + rr;
-              srow_i = (up ? rows_per_item : 0) + rr;
-            } else {
-              grow = r0 + r;
-              srow_i = r;
+            const int s = cnt % nstage;
+            if (!mbar_wait(&empty[s], ((cnt / nstage) & 1u) ^ 1u)) {
+              *s_abort = 1;
+              break;
             }
-            bulk_g2s_hint(sw_base + srow_i * SW, it.wbase + (int64_t)grow * row_bytes + kb, wbytes, &full[s], pol);
+            uint8_t* st_w = s_stage + s * STAGE_BYTES;
+            uint8_t* st_x = st_w + W_BYTES;
+            const int kb = ch * kLine;                 // byte offset inside a weight row
+            const int xb0 = ch * KC * 2;               // byte offset inside an activation row
+            int nxb = 0;
+            for (int q = 0; q < NXBOX; ++q) nxb += (xb0 + q * kLine < x_row_bytes) ? 1 : 0;
+            const uint32_t bytes =
+                it.valid ? (uint32_t)(nbox_w * kBoxRows * kLine + nxb * XCOLS * kLine) : 0u;
+            mbar_arrive_expect_tx(&full[s], bytes);
+            if (it.valid) {
+              if (kGateUp) {
+                tma_load_3d(st_w, tw, kb, r0, it.phys, &full[s], pol_w);
+                tma_load_3d(st_w + kBoxRows * kLine, tw, kb, a.N + r0, it.phys, &full[s], pol_w);
+              } else {
+                tma_load_3d(st_w, tw, kb, r0, it.phys, &full[s], pol_w);
+                if (nbox_w == 2) tma_load_3d(st_w + kBoxRows * kLine, tw, kb, r0 + kBoxRows, it.phys, &full[s], pol_w);
+              }
+              for (int q = 0; q < nxb; ++q)
+                tma_load_2d(st_x + q * XCOLS * kLine, &a.tm_x, xb0 + q * kLine, it.xrow0 + c0, &full[s], pol_x);
+            }
+            ++cnt;
           }
-          uint8_t* sx_base = sw_base + stage_w_bytes;
-          for (int j = lane; j < ncols; j += 32) {
-            int src;
-            if (kGateUp)
-              src = it.shared_idx >= 0 ? (c0 + j) : __ldg(a.row_token + it.row_start + c0 + j);
-            else
-              src = it.shared_idx >= 0 ? (a.T * a.k + it.shared_idx * a.T + c0 + j) : (it.row_start + c0 + j);
-            bulk_g2s(sx_base + j * SX, a.xsrc + ((int64_t)src * K + (int64_t)ch * KC) * 2, xbytes, &full[s]);
-          }
-          ++cnt;
         }
-        if (*s_abort) break;
       }
-      if (*s_abort) break;
-    }
-    // Let every copy this warp issued land before the block can exit.
-    if (lane == 0) {
+      // Let every load this lane issued land before the block can exit.
       const uint32_t first = cnt > (uint32_t)nstage ? cnt - nstage : 0;
       for (uint32_t c = first; c < cnt; ++c) mbar_wait(&full[c % nstage], (c / nstage) & 1u);
     }
@@ -261,12 +253,13 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const FfnArgs a
 
   // ======================================================= consumer warps
   const int g = lane >> 2, c = lane & 3;
+  const int sg = sigma8(g);
   uint32_t cnt = 0;
   int item_no = 0;
   const uint32_t stage0 = smem_u32(s_stage);
   const uint32_t scale0 = smem_u32(s_scale);
   for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++item_no) {
-    const Item it = decode_item<F, kGateUp>(a, item, ntile, n_act, s_act, s_offs);
+    const Item it = decode_item<F>(a, item, ntile, s_act, s_offs);
     const int r0 = it.tile * rows_per_item;
     const int nrows = min(rows_per_item, a.N - r0);
     const int passes = it.valid ? ceil_div(it.n_cols, XCOLS) : 0;
@@ -294,11 +287,13 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const FfnArgs a
       float tmp[NG][2][4];  // INT4 group partials
       for (int ch = 0; ch < nchunks; ++ch) {
         const int s = cnt % nstage;
-        if (!mbar_wait(&full[s], (cnt / nstage) & 1u)) *s_abort = 1;
-        if (*s_abort) break;
+        if (*s_abort || !mbar_wait(&full[s], (cnt / nstage) & 1u)) {
+          *s_abort = 1;
+          break;
+        }
         if (active && ncols > 0) {
-          const uint32_t wst = stage0 + s * stage_bytes;
-          const uint32_t xst = wst + stage_w_bytes;
+          const uint32_t wst = stage0 + s * STAGE_BYTES;
+          const uint32_t xst = wst + W_BYTES;
           const int nblk = min(KC, K - ch * KC) / 32;
 #pragma unroll 2
           for (int b = 0; b < nblk; ++b) {
@@ -307,8 +302,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const FfnArgs a
 #pragma unroll
               for (int mt = 0; mt < 2; ++mt) {
                 const int mr = mt ? m1 : m0;
-                const uint4 lo = lds128(wst + (mr + g) * SW + b * 64 + 16 * c);
-                const uint4 hi = lds128(wst + (mr + g + 8) * SW + b * 64 + 16 * c);
+                const uint32_t gran = (uint32_t)((4 * b + c) ^ sg) << 4;
+                const uint4 lo = lds128(wst + (mr + sg) * kLine + gran);
+                const uint4 hi = lds128(wst + (mr + 8 + sg) * kLine + gran);
                 A[mt][0][0] = lo.x; A[mt][0][1] = hi.x; A[mt][0][2] = lo.y; A[mt][0][3] = hi.y;
                 A[mt][1][0] = lo.z; A[mt][1][1] = hi.z; A[mt][1][2] = lo.w; A[mt][1][3] = hi.w;
               }
@@ -316,8 +312,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const FfnArgs a
 #pragma unroll
               for (int mt = 0; mt < 2; ++mt) {
                 const int mr = mt ? m1 : m0;
-                const uint32_t wlo = lds32(wst + (mr + g) * SW + b * 16 + 4 * c);
-                const uint32_t whi = lds32(wst + (mr + g + 8) * SW + b * 16 + 4 * c);
+                const uint32_t off = ((uint32_t)(b ^ g) << 4) + 4 * c;
+                const uint32_t wlo = lds32(wst + (mr + g) * kLine + off);
+                const uint32_t whi = lds32(wst + (mr + g + 8) * kLine + off);
                 uint32_t l0, l1, l2, l3, h0, h1, h2, h3;
                 if constexpr (F == kINT4) {
                   int4x8_to_f16x8(wlo, l0, l1, l2, l3);
@@ -349,10 +346,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const FfnArgs a
                 sc[mt][1] = e8m0_to_f32(lds8(sc_base + (mr + g + 8) * srow + blk));
               }
             }
-            const bool grp_first = (F == kINT4) && ((b & 3) == 0);
-            const bool grp_last = (F == kINT4) && (((b & 3) == 3) || (b == nblk - 1));
             if constexpr (F == kINT4) {
-              if (grp_first) {
+              if ((b & 3) == 0) {
 #pragma unroll
                 for (int q = 0; q < NG; ++q)
 #pragma unroll
@@ -361,10 +356,13 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const FfnArgs a
                     for (int r = 0; r < 4; ++r) tmp[q][mt][r] = 0.f;
               }
             }
+            // activation fragment address: box b/2, granule (b&1)*4+c of row q*8+sigma(g)
+            const uint32_t xoff = (uint32_t)(b >> 1) * (XCOLS * kLine) + (uint32_t)sg * kLine +
+                                  ((uint32_t)((((b & 1) << 2) + c) ^ sg) << 4);
 #pragma unroll
             for (int q = 0; q < NG; ++q) {
               if (q < ng_act) {
-                const uint4 xv = lds128(xst + (q * 8 + g) * SX + b * 64 + 16 * c);
+                const uint4 xv = lds128(xst + xoff + q * 8 * kLine);
 #pragma unroll
                 for (int mt = 0; mt < 2; ++mt) {
                   if constexpr (F == kMXFP4) {
@@ -389,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const FfnArgs a
               }
             }
             if constexpr (F == kINT4) {
-              if (grp_last) {
+              if ((b & 3) == 3 || b == nblk - 1) {
                 const int grp = (ch * KC + b * 32) / 128;
 #pragma unroll
                 for (int mt = 0; mt < 2; ++mt) {
@@ -420,36 +418,31 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const FfnArgs a
           if (q < ng_act) {
 #pragma unroll
             for (int hc = 0; hc < 2; ++hc) {
-              const int col = c0 + q * 8 + 2 * c + hc;
+              const int col = c0 + q * 8 + sigma8(2 * c + hc);  // activation row inside the expert
               if (col < it.n_cols) {
+                const int xrow = it.xrow0 + col;
                 float f = it.gscale;
-                if (F != kBF16) {
-                  int src;
-                  if (kGateUp)
-                    src = it.shared_idx >= 0 ? col : __ldg(a.row_token + it.row_start + col);
-                  else
-                    src = it.shared_idx >= 0 ? (a.T * a.k + it.shared_idx * a.T + col) : (it.row_start + col);
-                  f = ldexpf(f, __ldg(a.xexp + src));
-                }
+                if (F != kBF16) f = ldexpf(f, __ldg(a.xexp + xrow));
+                // weight rows held by this lane: (row g, row g+8) of each m-tile (bf16: sigma(g))
+                const int wr = (F == kBF16) ? sg : g;
                 if (kGateUp) {
-                  const int orow = it.shared_idx >= 0 ? (a.T * a.k + it.shared_idx * a.T + col) : (it.row_start + col);
-                  __nv_bfloat16* o = a.out_routed + (int64_t)orow * a.N + r0 + warp * 16;
+                  __nv_bfloat16* o = a.out_routed + (int64_t)xrow * a.N + r0 + warp * 16;
 #pragma unroll
                   for (int hr = 0; hr < 2; ++hr) {
                     const float gt = acc[q][0][hr * 2 + hc] * f;
                     const float up = acc[q][1][hr * 2 + hc] * f;
                     const float h = gt / (1.f + expf(-gt)) * up;
-                    o[g + 8 * hr] = __float2bfloat16_rn(h);
+                    o[wr + 8 * hr] = __float2bfloat16_rn(h);
                   }
                 } else {
                   __nv_bfloat16* o = it.shared_idx >= 0
                                          ? a.out_shared + ((int64_t)it.shared_idx * a.T + col) * a.N
-                                         : a.out_routed + (int64_t)(it.row_start + col) * a.N;
+                                         : a.out_routed + (int64_t)xrow * a.N;
 #pragma unroll
                   for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
                     for (int hr = 0; hr < 2; ++hr)
-                      o[r0 + warp * 32 + mt * 16 + g + 8 * hr] = __float2bfloat16_rn(acc[q][mt][hr * 2 + hc] * f);
+                      o[r0 + warp * 32 + mt * 16 + wr + 8 * hr] = __float2bfloat16_rn(acc[q][mt][hr * 2 + hc] * f);
                 }
               }
             }
@@ -466,16 +459,15 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const FfnArgs a
 }
 
 // ------------------------------------------------------------------ host side
-struct FfnLaunch {
-  int F, NG;
-  bool gate_up;
-};
-
 template <int F, int NG, bool GU>
 static cudaError_t launch_one(const FfnArgs& a, int grid, size_t smem, cudaStream_t st) {
   auto kern = ffn_stream_kernel<F, NG, GU>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (err != cudaSuccess) return err;
+  static thread_local int configured_smem = -1;
+  if (configured_smem != (int)smem) {
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    configured_smem = (int)smem;
+  }
   ProfScope prof(GU ? "ffn_stage1_gate_up" : "ffn_stage2_down", st);
   kern<<<grid, kThreads, smem, st>>>(a);
   return cudaGetLastError();
@@ -491,7 +483,6 @@ static cudaError_t dispatch_ng(const FfnArgs& a, int ng, int grid, size_t smem, 
 }
 
 static int fmt_kc(int F) { return F == kBF16 ? 64 : 256; }
-static int fmt_sw(int F) { return F == kBF16 ? 192 : 144; }
 static int fmt_srow(int F, int K) {
   switch (F) {
     case kMXFP4: return K / 32;
@@ -503,28 +494,28 @@ static int fmt_srow(int F, int K) {
 
 // Shared memory plan of one stage kernel; returns false when it cannot fit.
 static bool plan_smem(int F, int ng, int K, int E, int smem_max, FfnArgs& a, size_t& total) {
-  const int hdr = ((16 * kMaxStages + 32 + 16 + 8 * E + 64) + 127) & ~127;
-  const int sbuf = ((kRowsPerTile * fmt_srow(F, K)) + 127) & ~127;
-  const int stage = kRowsPerTile * fmt_sw(F) + ng * 8 * (fmt_kc(F) * 2 + 64);
+  const int hdr = ((16 * kMaxStages + 32 + 16 + 8 * E + 64) + 1023) & ~1023;
+  const int sbuf = ((kRowsPerStage * fmt_srow(F, K)) + 1023) & ~1023;
+  const int stage = kRowsPerStage * kLine + ((fmt_kc(F) * 2) / kLine) * ng * 8 * kLine;
+  const int usable = smem_max - 1024;  // room for the runtime 1024-byte alignment
   for (int nsb = 2; nsb >= 1; --nsb) {
-    if (F == kBF16 && nsb == 2) continue;
     const int nsbx = (F == kBF16) ? 1 : nsb;
-    const int room = smem_max - hdr - nsbx * sbuf;
+    const int room = usable - hdr - nsbx * sbuf;
     int ns = room / stage;
     if (ns > kMaxStages) ns = kMaxStages;
     if (ns >= 3 || (nsb == 1 && ns >= 2)) {
       a.n_stages = ns;
       a.n_scale_buf = nsbx;
       a.smem_scale_bytes = sbuf;
-      total = (size_t)hdr + (size_t)nsbx * sbuf + (size_t)ns * stage;
+      total = (size_t)1024 + hdr + (size_t)nsbx * sbuf + (size_t)ns * stage;
       return true;
     }
   }
   return false;
 }
 
-cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, int T, int n_sms, int smem_max, cudaStream_t st,
-                              int* unsupported) {
+cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers& p, int T, int n_sms,
+                              int smem_max, cudaStream_t st, int* unsupported) {
   *unsupported = 0;
   const int ng = T <= 8 ? 1 : (T <= 16 ? 2 : 4);
   size_t smem = 0;
@@ -532,7 +523,39 @@ cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, int T, int n_sms, 
     *unsupported = 1;
     return cudaSuccess;
   }
-  const int rows_per_item = gate_up ? kRowsPerTile / 2 : kRowsPerTile;
+  // tensor maps
+  const uint64_t row_bytes = (F == kBF16) ? (uint64_t)a.K * 2 : (uint64_t)a.K / 2;
+  const uint64_t wrows = gate_up ? 2 * (uint64_t)a.N : (uint64_t)a.N;
+  {
+    const uint64_t dims[3] = {row_bytes, wrows, (uint64_t)a.n_phys};
+    const uint64_t strides[2] = {row_bytes, (uint64_t)p.stride_w};
+    const uint32_t box[3] = {kLine, kBoxRows, 1};
+    if (!encode_tmap_u8(&a.tm_w, p.w, 3, dims, strides, box, true)) {
+      *unsupported = 1;
+      return cudaSuccess;
+    }
+  }
+  if (a.n_shared > 0) {
+    const uint64_t dims[3] = {row_bytes, wrows, (uint64_t)a.n_shared};
+    const uint64_t strides[2] = {row_bytes, (uint64_t)p.stride_w_sh};
+    const uint32_t box[3] = {kLine, kBoxRows, 1};
+    if (!encode_tmap_u8(&a.tm_wsh, p.w_sh, 3, dims, strides, box, true)) {
+      *unsupported = 1;
+      return cudaSuccess;
+    }
+  } else {
+    a.tm_wsh = a.tm_w;
+  }
+  {
+    const uint64_t dims[2] = {(uint64_t)a.K * 2, (uint64_t)p.rows_total};
+    const uint64_t strides[1] = {(uint64_t)a.K * 2};
+    const uint32_t box[2] = {kLine, (uint32_t)(ng * 8)};
+    if (!encode_tmap_u8(&a.tm_x, p.x, 2, dims, strides, box, true)) {
+      *unsupported = 1;
+      return cudaSuccess;
+    }
+  }
+  const int rows_per_item = gate_up ? kRowsPerStage / 2 : kRowsPerStage;
   const int ntile = ceil_div(a.N, rows_per_item);
   const long max_items = (long)(a.n_shared + (a.E < T * a.k ? a.E : T * a.k)) * ntile;
   int grid = (int)(max_items < n_sms ? max_items : n_sms);

@@ -24,8 +24,8 @@ cudaError_t launch_route_topk(const moe_layer_desc& dsc, const void* x, const vo
                               float* logits, int32_t* topk_idx, float* topk_w, cudaStream_t st);
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* offsets, int32_t* row_token,
                            int32_t* inv, cudaStream_t st);
-cudaError_t launch_prep_rows(const void* src, int rows, int K, bool perm_int4, void* dst, int32_t* rexp,
-                             cudaStream_t st);
+cudaError_t launch_prep_rows(const void* src, int rows, int K, int mode, void* dst, int32_t* rexp,
+                             const int32_t* gather, int n_gather, int n_tok, cudaStream_t st);
 cudaError_t launch_combine(const void* y, const int32_t* inv, const float* gw, const void* y_shared, int n_shared,
                            int T, int d, int k, void* out, cudaStream_t st);
 
@@ -58,7 +58,7 @@ int64_t scale_bytes(int f, int64_t N, int64_t K) {
 }
 
 struct Layout {
-  size_t logits, topk_idx, topk_w, offsets, row_token, inv, xq, xexp, h, hq, hexp, y, ysh, total;
+  size_t logits, topk_idx, topk_w, offsets, row_token, inv, xperm, xexp, h, hq, hexp, y, ysh, total;
 };
 
 Layout layout_of(const moe_layer_desc& d) {
@@ -78,8 +78,8 @@ Layout layout_of(const moe_layer_desc& d) {
   L.row_token = take(R * 4);
   L.inv = take(R * 4);
   const bool q = is4bit(d.wdtype);
-  L.xq = take(q ? T * D * 2 : 0);
-  L.xexp = take(q ? T * 4 : 0);
+  L.xperm = take(RT * D * 2);
+  L.xexp = take(q ? RT * 4 : 0);
   L.h = take(RT * F * 2);
   L.hq = take(q ? RT * F * 2 : 0);
   L.hexp = take(q ? RT * 4 : 0);
@@ -149,38 +149,38 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
   const int R = T * k, RT = R + S * T;
   const DevInfo di = dev_info();
   cudaError_t err;
-  __half* xq = reinterpret_cast<__half*>(ws + L.xq);
+  void* xperm = ws + L.xperm;
   int32_t* xexp = reinterpret_cast<int32_t*>(ws + L.xexp);
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
   __half* hq = reinterpret_cast<__half*>(ws + L.hq);
   int32_t* hexp = reinterpret_cast<int32_t*>(ws + L.hexp);
-  if (q) {
-    err = launch_prep_rows(x, T, D, f == MOE_W_INT4_G128, xq, xexp, st);
-    if (err != cudaSuccess) return MOE_ERR_CUDA;
-  }
-  auto fill = [&](FfnArgs& a, bool stage1) {
+  const int mode = !q ? 2 : (f == MOE_W_INT4_G128 ? 1 : 0);
+  // activation rows in expert order (routed rows, then every token once per shared expert)
+  err = launch_prep_rows(x, RT, D, mode, xperm, xexp, row_token, R, T, st);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  auto fill = [&](FfnArgs& a, FfnPointers& p, bool stage1) {
     std::memset(&a, 0, sizeof(a));
+    std::memset(&p, 0, sizeof(p));
     const int64_t N = stage1 ? 2 * (int64_t)F : D, K = stage1 ? D : F;
-    const void* wv = stage1 ? routed->w13 : routed->w2;
-    const void* sv = stage1 ? routed->s13 : routed->s2;
-    int64_t sw = stage1 ? routed->stride_w13 : routed->stride_w2;
-    int64_t ss = stage1 ? routed->stride_s13 : routed->stride_s2;
-    a.w = static_cast<const uint8_t*>(wv);
-    a.s = static_cast<const uint8_t*>(sv);
-    a.gsc = stage1 ? routed->g13 : routed->g2;
-    a.stride_w = sw ? sw : mat_bytes(f, N, K);
+    const int64_t sw = stage1 ? routed->stride_w13 : routed->stride_w2;
+    const int64_t ss = stage1 ? routed->stride_s13 : routed->stride_s2;
+    p.w = stage1 ? routed->w13 : routed->w2;
+    p.stride_w = sw ? sw : mat_bytes(f, N, K);
+    a.s = static_cast<const uint8_t*>(stage1 ? routed->s13 : routed->s2);
     a.stride_s = ss ? ss : scale_bytes(f, N, K);
+    a.gsc = stage1 ? routed->g13 : routed->g2;
     a.slot_map = routed->slot_map;
     a.n_phys = routed->n_physical ? routed->n_physical : E;
     if (S > 0) {
-      a.w_sh = static_cast<const uint8_t*>(stage1 ? shared->w13 : shared->w2);
-      a.s_sh = static_cast<const uint8_t*>(stage1 ? shared->s13 : shared->s2);
-      a.gsc_sh = stage1 ? shared->g13 : shared->g2;
       const int64_t shw = stage1 ? shared->stride_w13 : shared->stride_w2;
       const int64_t shs = stage1 ? shared->stride_s13 : shared->stride_s2;
-      a.stride_w_sh = shw ? shw : mat_bytes(f, N, K);
+      p.w_sh = stage1 ? shared->w13 : shared->w2;
+      p.stride_w_sh = shw ? shw : mat_bytes(f, N, K);
+      a.s_sh = static_cast<const uint8_t*>(stage1 ? shared->s13 : shared->s2);
       a.stride_s_sh = shs ? shs : scale_bytes(f, N, K);
+      a.gsc_sh = stage1 ? shared->g13 : shared->g2;
     }
+    p.rows_total = RT;
     a.n_shared = S;
     a.E = E;
     a.T = T;
@@ -188,29 +188,30 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
     a.N = stage1 ? F : D;
     a.K = (int)K;
     a.offsets = offsets;
-    a.row_token = row_token;
   };
   FfnArgs a1;
-  fill(a1, true);
-  a1.xsrc = static_cast<const uint8_t*>(q ? static_cast<const void*>(xq) : x);
+  FfnPointers p1;
+  fill(a1, p1, true);
+  p1.x = xperm;
   a1.xexp = q ? xexp : nullptr;
   a1.out_routed = h;
   a1.out_shared = nullptr;
   int unsup = 0;
-  err = launch_ffn_stream(f, true, a1, T, di.sms, di.smem_optin, st, &unsup);
+  err = launch_ffn_stream(f, true, a1, p1, T, di.sms, di.smem_optin, st, &unsup);
   if (unsup) return MOE_ERR_UNSUPPORTED;
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   if (q) {
-    err = launch_prep_rows(h, RT, F, f == MOE_W_INT4_G128, hq, hexp, st);
+    err = launch_prep_rows(h, RT, F, mode, hq, hexp, nullptr, 0, T, st);
     if (err != cudaSuccess) return MOE_ERR_CUDA;
   }
   FfnArgs a2;
-  fill(a2, false);
-  a2.xsrc = reinterpret_cast<const uint8_t*>(q ? static_cast<void*>(hq) : static_cast<void*>(h));
+  FfnPointers p2;
+  fill(a2, p2, false);
+  p2.x = q ? static_cast<const void*>(hq) : static_cast<const void*>(h);
   a2.xexp = q ? hexp : nullptr;
   a2.out_routed = static_cast<__nv_bfloat16*>(y_perm);
   a2.out_shared = static_cast<__nv_bfloat16*>(y_shared);
-  err = launch_ffn_stream(f, false, a2, T, di.sms, di.smem_optin, st, &unsup);
+  err = launch_ffn_stream(f, false, a2, p2, T, di.sms, di.smem_optin, st, &unsup);
   if (unsup) return MOE_ERR_UNSUPPORTED;
   return from_cuda(err);
 }

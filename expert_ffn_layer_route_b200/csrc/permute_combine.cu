@@ -106,21 +106,33 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* off
 }
 
 // ---------------------------------------------------------------------------
-// Activation rows -> fp16 for the 4-bit weight paths.  Each row is scaled by
-// 2^-p with p = floor(log2(max|row|)) - 14 so that its largest magnitude lies
-// in [2^14, 2^15) (fp16's range); rexp[row] = p is undone on the accumulators.
-// With kPermInt4 each 8-element group is stored in the order
-// 0,4,1,5,2,6,3,7, the pairing the INT4 decoder produces.
+// Activation rows for the grouped FFN, written in expert order so that an
+// expert's rows are contiguous.  Output row r reads source row gather[r] for
+// r < n_gather and row (r - n_gather) % n_tok after that (the shared experts'
+// copies of every token); with no gather array, row r reads row r.
+// Modes: kCopyBf16 copies the bf16 row; otherwise the row is converted to fp16
+// after scaling by 2^-p with p = floor(log2(max|row|)) - 14, so that its
+// largest magnitude lies in [2^14, 2^15) (fp16's range), and rexp[r] = p is
+// undone on the accumulators.  kPermInt4 stores each 8-element group in the
+// order 0,4,1,5,2,6,3,7, the pairing the INT4 decoder produces.
 constexpr int kPrepThreads = 128;
+enum PrepMode : int { kF16 = 0, kF16PermInt4 = 1, kCopyBf16 = 2 };
 
-template <bool kPermInt4>
+template <int kMode>
 __global__ void __launch_bounds__(kPrepThreads)
-    prep_rows_kernel(const __nv_bfloat16* __restrict__ src, int K, __half* __restrict__ dst,
-                     int32_t* __restrict__ rexp) {
+    prep_rows_kernel(const __nv_bfloat16* __restrict__ src, int K, void* __restrict__ dst,
+                     int32_t* __restrict__ rexp, const int32_t* __restrict__ gather, int n_gather, int n_tok) {
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
-  const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)row * K);
+  int srow = row;
+  if (gather) srow = row < n_gather ? __ldg(gather + row) : (row - n_gather) % n_tok;
+  const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)srow * K);
   const int nchunk = K / 8;
+  if constexpr (kMode == kCopyBf16) {
+    uint4* d = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + (size_t)row * K);
+    for (int c = tid; c < nchunk; c += kPrepThreads) d[c] = __ldg(s + c);
+    return;
+  }
   float amax = 0.f;
   for (int c = tid; c < nchunk; c += kPrepThreads) {
     const uint4 u = __ldg(s + c);
@@ -147,7 +159,7 @@ __global__ void __launch_bounds__(kPrepThreads)
   }
   if (tid == 0) rexp[row] = p;
   const float scale = ldexpf(1.f, -p);
-  uint4* d = reinterpret_cast<uint4*>(dst + (size_t)row * K);
+  uint4* d = reinterpret_cast<uint4*>(static_cast<__half*>(dst) + (size_t)row * K);
   for (int c = tid; c < nchunk; c += kPrepThreads) {
     const uint4 u = __ldg(s + c);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -158,7 +170,7 @@ __global__ void __launch_bounds__(kPrepThreads)
       f[2 * q + 1] = bf16_bits_to_f32(w[q] >> 16) * scale;
     }
     __half h[8];
-    if (kPermInt4) {
+    if constexpr (kMode == kF16PermInt4) {
       const int order[8] = {0, 4, 1, 5, 2, 6, 3, 7};
 #pragma unroll
       for (int q = 0; q < 8; ++q) h[q] = __float2half_rn(f[order[q]]);
@@ -170,16 +182,18 @@ __global__ void __launch_bounds__(kPrepThreads)
   }
 }
 
-cudaError_t launch_prep_rows(const void* src, int rows, int K, bool perm_int4, void* dst, int32_t* rexp,
-                             cudaStream_t st) {
+// mode: 0 fp16 scaled, 1 fp16 scaled in INT4 pairing order, 2 bf16 copy.
+cudaError_t launch_prep_rows(const void* src, int rows, int K, int mode, void* dst, int32_t* rexp,
+                             const int32_t* gather, int n_gather, int n_tok, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  ProfScope prof("prep_rows", st);
-  if (perm_int4)
-    prep_rows_kernel<true><<<rows, kPrepThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(src), K,
-                                                          static_cast<__half*>(dst), rexp);
+  ProfScope prof(gather ? "prep_x_gather" : "prep_h", st);
+  const __nv_bfloat16* s = static_cast<const __nv_bfloat16*>(src);
+  if (mode == kCopyBf16)
+    prep_rows_kernel<kCopyBf16><<<rows, kPrepThreads, 0, st>>>(s, K, dst, rexp, gather, n_gather, n_tok);
+  else if (mode == kF16PermInt4)
+    prep_rows_kernel<kF16PermInt4><<<rows, kPrepThreads, 0, st>>>(s, K, dst, rexp, gather, n_gather, n_tok);
   else
-    prep_rows_kernel<false><<<rows, kPrepThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(src), K,
-                                                           static_cast<__half*>(dst), rexp);
+    prep_rows_kernel<kF16><<<rows, kPrepThreads, 0, st>>>(s, K, dst, rexp, gather, n_gather, n_tok);
   return cudaGetLastError();
 }
 
