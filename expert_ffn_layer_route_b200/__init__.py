@@ -23,6 +23,7 @@ from ._native import (  # noqa: F401
     moe_workspace_size,
     moe_workspace_layout_of,
     moe_route_topk,
+    moe_route_topk_noalloc,
     moe_permute,
     moe_grouped_ffn,
     moe_combine,

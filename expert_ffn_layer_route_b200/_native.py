@@ -68,6 +68,7 @@ _SIGS = {
     "moe_workspace_size": [_DP, ctypes.POINTER(ctypes.c_size_t)],
     "moe_workspace_layout_of": [_DP, ctypes.POINTER(WorkspaceLayout)],
     "moe_route_topk": [_DP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+    "moe_route_topk_noalloc": [_DP, _P, _P, _P, _P, _P, _P],
     "moe_permute": [_DP, _P, _P, _P, _P, _P],
     "moe_grouped_ffn": [_DP, _WP, _WP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "moe_combine": [_DP, _P, _P, _P, _P, _P, _P],
@@ -178,6 +179,12 @@ def moe_route_topk(desc, x, w_router, logit_bias, topk_idx, topk_w, workspace, s
     _check(lib().moe_route_topk(ctypes.byref(desc), _ptr(x), _ptr(w_router), _ptr(logit_bias), _ptr(topk_idx),
                                 _ptr(topk_w), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                 _stream(stream)), "moe_route_topk")
+
+
+def moe_route_topk_noalloc(desc, x, w_router, logit_bias, topk_idx, topk_w, stream=None):
+    """moe_route_topk with the library's fixed scratch (for callers that cannot allocate)."""
+    _check(lib().moe_route_topk_noalloc(ctypes.byref(desc), _ptr(x), _ptr(w_router), _ptr(logit_bias),
+                                        _ptr(topk_idx), _ptr(topk_w), _stream(stream)), "moe_route_topk_noalloc")
 
 
 def moe_permute(desc, topk_idx, offsets, row_token, inv, stream=None):

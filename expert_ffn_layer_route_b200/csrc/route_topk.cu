@@ -18,6 +18,8 @@
 //
 // Kernel 2 (topk_kernel): one warp per token.  k rounds of a warp-wide
 // argmax over (logit desc, index asc); gates from expf in fp32.
+#include <mutex>
+
 #include "common.cuh"
 #include "profile.cuh"
 
@@ -182,3 +184,61 @@ cudaError_t launch_route_topk(const moe_layer_desc& dsc, const void* x, const vo
 }
 
 }  // namespace moe
+
+// ---------------------------------------------------------------------------
+// Router + top-k for callers that cannot allocate device memory.
+//
+// moe_route_topk takes its logits scratch from a caller-provided workspace.
+// Some callers have no way to provide one: plugins whose host framework owns
+// every device allocation and hands them none, runtimes that fix their device
+// memory at start-up and forbid allocation afterwards, code on paths where a
+// device allocation would synchronise or fail.  For them the logits live in a
+// fixed file-scope device array instead, sized for T * n_experts <= 262144
+// (1 MiB of fp32); every GPU that loads this library holds it until exit.
+//
+// Host code must not pass the array's name to a kernel: on the host it is a
+// stand-in symbol, not a device address.  The device address is looked up
+// once per device with cudaGetSymbolAddress on the first call made with that
+// device current, so that first call should come before any stream capture.
+// All calls share the one array: calls that overlap on the GPU (different
+// streams, no ordering between them) race on it.  Nothing in it needs to
+// start at zero: each call writes every logit it later reads.
+namespace {
+
+constexpr size_t kNoAllocLogitsMax = 262144;
+__device__ __align__(256) float g_noalloc_logits[kNoAllocLogitsMax];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+}  // namespace
+
+extern "C" moe_status moe_route_topk_noalloc(const moe_layer_desc* desc, const void* x, const void* w_router,
+                                             const float* logit_bias, int32_t* topk_idx, float* topk_w,
+                                             void* stream) {
+  size_t ws_bytes = 0;
+  moe_status s = moe_workspace_size(desc, &ws_bytes);  // validates the descriptor
+  if (s != MOE_OK) return s;
+  if (desc->T == 0) return MOE_OK;
+  if (!x || !w_router || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(w_router)) & 15u) return MOE_ERR_INVALID_ARG;
+  if ((size_t)desc->T * (size_t)desc->n_experts > kNoAllocLogitsMax) return MOE_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return MOE_ERR_UNSUPPORTED;
+  float* logits = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_logits) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+      g_noalloc_ptr[dev] = static_cast<float*>(p);
+    }
+    logits = g_noalloc_ptr[dev];
+  }
+  return moe::launch_route_topk(*desc, x, w_router, logit_bias, logits, topk_idx, topk_w,
+                                static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}

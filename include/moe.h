@@ -147,6 +147,20 @@ moe_status moe_route_topk(const moe_layer_desc* desc, const void* x, const void*
                           const float* logit_bias, int32_t* topk_idx, float* topk_w,
                           void* workspace, size_t ws_bytes, void* stream);
 
+/* moe_route_topk for callers that cannot allocate device memory (no
+ * counterpart in the paper: an interface convenience of this library).
+ * Same inputs, outputs and arithmetic as moe_route_topk, but the fp32 logits
+ * scratch is a fixed device array inside the library instead of a caller
+ * workspace: for plugins whose host framework owns every device allocation,
+ * or runtimes that fix their device memory at start-up.  Limit: T * n_experts
+ * <= 262144 (1 MiB, held on every GPU that loads the library until exit);
+ * larger calls return MOE_ERR_WORKSPACE before enqueueing anything.  The
+ * first call on a device looks up the array's device address (make it before
+ * any stream capture).  Calls share the array: calls that overlap on the GPU
+ * race.  Nothing is allocated. */
+moe_status moe_route_topk_noalloc(const moe_layer_desc* desc, const void* x, const void* w_router,
+                                  const float* logit_bias, int32_t* topk_idx, float* topk_w, void* stream);
+
 /* Stable counting sort of the T*k (token, slot) pairs by expert.
  * offsets int32 [E+1] (exclusive prefix sum of per-expert counts),
  * row_token int32 [T*k] (token of each grouped row; rows of one expert are in
