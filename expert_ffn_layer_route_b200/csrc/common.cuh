@@ -171,6 +171,27 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
   return *reinterpret_cast<uint32_t*>(&r);
 }
 
+// Two E8M0 scales (low byte, high byte of a 16-bit value) -> two fp32 values
+// 2^(v-127), exact (v = 0 gives 2^-127, v = 255 NaN), via the hardware
+// conversion to bf16x2 (same exponent range as fp32) and a shift.
+__device__ __forceinline__ void e8m0x2_to_f32x2(uint32_t pair16, float& lo, float& hi) {
+  uint32_t b2;
+  asm("{\n .reg .b16 t;\n cvt.u16.u32 t, %1;\n cvt.rn.bf16x2.ue8m0x2 %0, t;\n}\n" : "=r"(b2) : "r"(pair16));
+  lo = __uint_as_float(b2 << 16);
+  hi = __uint_as_float(b2 & 0xffff0000u);
+}
+
+// D = A * B (accumulator starts at zero).
+__device__ __forceinline__ void mma_f16_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  const float z = 0.f;
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
+}
+
 // E8M0 byte -> fp32 2^(v-127) (v = 255 -> NaN).
 __device__ __forceinline__ float e8m0_to_f32(uint32_t v) {
   if (v == 0u) return __int_as_float(0x00400000);  // 2^-127 (subnormal)

@@ -29,6 +29,8 @@
 // weight rows) are read through the row order sigma(g) = (g>>1) | (g&1)<<2
 // inside each group of 8 so that the swizzled 16-byte reads are free of bank
 // conflicts; the epilogue maps columns (rows) back through the same sigma.
+#include <cstdlib>
+
 #include "ffn_stream.cuh"
 #include "profile.cuh"
 
@@ -111,8 +113,8 @@ __device__ __forceinline__ Item decode_item(const FfnArgs& a, int item, int ntil
   return it;
 }
 
-template <int F, int NG, bool kGateUp>
-__global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const __grid_constant__ FfnArgs a) {
+template <int F, int NG, bool kGateUp, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid_constant__ FfnArgs a) {
   using Tr = FmtTraits<F>;
   constexpr int KC = Tr::kc;
   constexpr int XCOLS = NG * 8;                 // activation rows per pass
@@ -295,8 +297,28 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const __grid_co
           const uint32_t wst = stage0 + s * STAGE_BYTES;
           const uint32_t xst = wst + W_BYTES;
           const int nblk = min(KC, K - ch * KC) / 32;
-#pragma unroll 2
-          for (int b = 0; b < nblk; ++b) {
+          // 32-wide K blocks in pairs: the MXFP4 scales of a pair load as one
+          // 16-bit value per row (low byte: even block)
+          const bool pair_aligned = (srow & 1) == 0;
+          for (int bp = 0; bp < nblk; bp += 2) {
+            float scp[2][2][2];  // MXFP4 scales [m-tile][row g / g+8][block of the pair]
+            if constexpr (F == kMXFP4) {
+              const int blk = (ch * KC) / 32 + bp;
+#pragma unroll
+              for (int mt = 0; mt < 2; ++mt) {
+                const int mr = mt ? m1 : m0;
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {
+                  const uint32_t ad = sc_base + (mr + g + 8 * hr) * srow + blk;
+                  const uint32_t v = pair_aligned ? lds16(ad) : (lds8(ad) | (lds8(ad + 1) << 8));
+                  e8m0x2_to_f32x2(v, scp[mt][hr][0], scp[mt][hr][1]);
+                }
+              }
+            }
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb) {
+            const int b = bp + hb;
+            if (b >= nblk) break;
             uint32_t A[2][2][4];  // [m-tile][k16 tile][reg]
             if constexpr (F == kBF16) {
 #pragma unroll
@@ -336,16 +358,6 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const __grid_co
                 A[mt][1][0] = l2; A[mt][1][1] = h2; A[mt][1][2] = l3; A[mt][1][3] = h3;
               }
             }
-            float sc[2][2];
-            if constexpr (F == kMXFP4) {
-              const int blk = (ch * KC) / 32 + b;
-#pragma unroll
-              for (int mt = 0; mt < 2; ++mt) {
-                const int mr = mt ? m1 : m0;
-                sc[mt][0] = e8m0_to_f32(lds8(sc_base + (mr + g) * srow + blk));
-                sc[mt][1] = e8m0_to_f32(lds8(sc_base + (mr + g + 8) * srow + blk));
-              }
-            }
             if constexpr (F == kINT4) {
               if ((b & 3) == 0) {
 #pragma unroll
@@ -358,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const __grid_co
             }
             // activation fragment address: box b/2, granule (b&1)*4+c of row q*8+sigma(g)
             const uint32_t xoff = (uint32_t)(b >> 1) * (XCOLS * kLine) + (uint32_t)sg * kLine +
-                                  ((uint32_t)((((b & 1) << 2) + c) ^ sg) << 4);
+                                  ((uint32_t)(((hb << 2) + c) ^ sg) << 4);
 #pragma unroll
             for (int q = 0; q < NG; ++q) {
               if (q < ng_act) {
@@ -366,13 +378,13 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const __grid_co
 #pragma unroll
                 for (int mt = 0; mt < 2; ++mt) {
                   if constexpr (F == kMXFP4) {
-                    float t4[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma_f16(t4, A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
+                    float t4[4];
+                    mma_f16_z(t4, A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
                     mma_f16(t4, A[mt][1][0], A[mt][1][1], A[mt][1][2], A[mt][1][3], xv.z, xv.w);
-                    acc[q][mt][0] = fmaf(t4[0], sc[mt][0], acc[q][mt][0]);
-                    acc[q][mt][1] = fmaf(t4[1], sc[mt][0], acc[q][mt][1]);
-                    acc[q][mt][2] = fmaf(t4[2], sc[mt][1], acc[q][mt][2]);
-                    acc[q][mt][3] = fmaf(t4[3], sc[mt][1], acc[q][mt][3]);
+                    acc[q][mt][0] = fmaf(t4[0], scp[mt][0][hb], acc[q][mt][0]);
+                    acc[q][mt][1] = fmaf(t4[1], scp[mt][0][hb], acc[q][mt][1]);
+                    acc[q][mt][2] = fmaf(t4[2], scp[mt][1][hb], acc[q][mt][2]);
+                    acc[q][mt][3] = fmaf(t4[3], scp[mt][1][hb], acc[q][mt][3]);
                   } else if constexpr (F == kINT4) {
                     mma_f16(tmp[q][mt], A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
                     mma_f16(tmp[q][mt], A[mt][1][0], A[mt][1][1], A[mt][1][2], A[mt][1][3], xv.z, xv.w);
@@ -403,6 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const __grid_co
                   }
                 }
               }
+            }
             }
           }
         }
@@ -459,9 +472,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_stream_kernel(const __grid_co
 }
 
 // ------------------------------------------------------------------ host side
-template <int F, int NG, bool GU>
+template <int F, int NG, bool GU, int MINB>
 static cudaError_t launch_one(const FfnArgs& a, int grid, size_t smem, cudaStream_t st) {
-  auto kern = ffn_stream_kernel<F, NG, GU>;
+  auto kern = ffn_stream_kernel<F, NG, GU, MINB>;
   static thread_local int configured_smem = -1;
   if (configured_smem != (int)smem) {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -474,11 +487,17 @@ static cudaError_t launch_one(const FfnArgs& a, int grid, size_t smem, cudaStrea
 }
 
 template <int F, bool GU>
-static cudaError_t dispatch_ng(const FfnArgs& a, int ng, int grid, size_t smem, cudaStream_t st) {
+static cudaError_t dispatch_ng(const FfnArgs& a, int ng, int minb, int grid, size_t smem, cudaStream_t st) {
+  if (minb == 2) {
+    switch (ng) {
+      case 1: return launch_one<F, 1, GU, 2>(a, grid, smem, st);
+      default: return launch_one<F, 2, GU, 2>(a, grid, smem, st);
+    }
+  }
   switch (ng) {
-    case 1: return launch_one<F, 1, GU>(a, grid, smem, st);
-    case 2: return launch_one<F, 2, GU>(a, grid, smem, st);
-    default: return launch_one<F, 4, GU>(a, grid, smem, st);
+    case 1: return launch_one<F, 1, GU, 1>(a, grid, smem, st);
+    case 2: return launch_one<F, 2, GU, 1>(a, grid, smem, st);
+    default: return launch_one<F, 4, GU, 1>(a, grid, smem, st);
   }
 }
 
@@ -515,11 +534,27 @@ static bool plan_smem(int F, int ng, int K, int E, int smem_max, FfnArgs& a, siz
 }
 
 cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers& p, int T, int n_sms,
-                              int smem_max, cudaStream_t st, int* unsupported) {
+                              int smem_max, int smem_per_sm, cudaStream_t st, int* unsupported) {
   *unsupported = 0;
-  const int ng = T <= 8 ? 1 : (T <= 16 ? 2 : 4);
+  // Columns per pass (NG groups of 8 activation rows) and CTAs per SM.  Two
+  // CTAs of 8 consumer warps hide the decode's fixed-latency dependencies
+  // better than one (measured on the gpt-oss decode batch: stage 1 at 4.2 vs
+  // 3.2 TB/s); 16 columns cover almost every routed expert of a decode batch
+  // in one pass.  MOE_FFN_NG / MOE_FFN_MINB override the choice for tuning.
+  int ng = T <= 8 ? 1 : 2;
+  int minb = 2;
+  if (const char* e = getenv("MOE_FFN_NG")) ng = atoi(e);
+  if (const char* e = getenv("MOE_FFN_MINB")) minb = atoi(e);
+  if (ng != 1 && ng != 2 && ng != 4) ng = 2;
+  if (minb == 2 && ng > 2) ng = 2;
   size_t smem = 0;
-  if (!plan_smem(F, ng, a.K, a.E, smem_max, a, smem)) {
+  bool ok = false;
+  if (minb == 2) ok = plan_smem(F, ng, a.K, a.E, smem_per_sm / 2 - 1024, a, smem);
+  if (!ok) {
+    minb = 1;
+    ok = plan_smem(F, ng, a.K, a.E, smem_max, a, smem);
+  }
+  if (!ok) {
     *unsupported = 1;
     return cudaSuccess;
   }
@@ -558,13 +593,14 @@ cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers&
   const int rows_per_item = gate_up ? kRowsPerStage / 2 : kRowsPerStage;
   const int ntile = ceil_div(a.N, rows_per_item);
   const long max_items = (long)(a.n_shared + (a.E < T * a.k ? a.E : T * a.k)) * ntile;
-  int grid = (int)(max_items < n_sms ? max_items : n_sms);
+  const long slots = (long)n_sms * minb;
+  int grid = (int)(max_items < slots ? max_items : slots);
   if (grid < 1) return cudaSuccess;
   switch (F) {
-    case kBF16: return gate_up ? dispatch_ng<kBF16, true>(a, ng, grid, smem, st) : dispatch_ng<kBF16, false>(a, ng, grid, smem, st);
-    case kMXFP4: return gate_up ? dispatch_ng<kMXFP4, true>(a, ng, grid, smem, st) : dispatch_ng<kMXFP4, false>(a, ng, grid, smem, st);
-    case kNVFP4: return gate_up ? dispatch_ng<kNVFP4, true>(a, ng, grid, smem, st) : dispatch_ng<kNVFP4, false>(a, ng, grid, smem, st);
-    default: return gate_up ? dispatch_ng<kINT4, true>(a, ng, grid, smem, st) : dispatch_ng<kINT4, false>(a, ng, grid, smem, st);
+    case kBF16: return gate_up ? dispatch_ng<kBF16, true>(a, ng, minb, grid, smem, st) : dispatch_ng<kBF16, false>(a, ng, minb, grid, smem, st);
+    case kMXFP4: return gate_up ? dispatch_ng<kMXFP4, true>(a, ng, minb, grid, smem, st) : dispatch_ng<kMXFP4, false>(a, ng, minb, grid, smem, st);
+    case kNVFP4: return gate_up ? dispatch_ng<kNVFP4, true>(a, ng, minb, grid, smem, st) : dispatch_ng<kNVFP4, false>(a, ng, minb, grid, smem, st);
+    default: return gate_up ? dispatch_ng<kINT4, true>(a, ng, minb, grid, smem, st) : dispatch_ng<kINT4, false>(a, ng, minb, grid, smem, st);
   }
 }
 

@@ -53,6 +53,6 @@ struct FfnPointers {
 };
 
 cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers& p, int T, int n_sms,
-                              int smem_max, cudaStream_t st, int* unsupported);
+                              int smem_max, int smem_per_sm, cudaStream_t st, int* unsupported);
 
 }  // namespace moe

@@ -105,7 +105,7 @@ moe_status check_desc(const moe_layer_desc* d) {
 }
 
 struct DevInfo {
-  int sms = 0, smem_optin = 0;
+  int sms = 0, smem_optin = 0, smem_per_sm = 0;
 };
 
 DevInfo dev_info() {
@@ -118,6 +118,7 @@ DevInfo dev_info() {
   if (cache[dev].sms == 0) {
     cudaDeviceGetAttribute(&cache[dev].sms, cudaDevAttrMultiProcessorCount, dev);
     cudaDeviceGetAttribute(&cache[dev].smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    cudaDeviceGetAttribute(&cache[dev].smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
   }
   return cache[dev];
 }
@@ -197,7 +198,7 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
   a1.out_routed = h;
   a1.out_shared = nullptr;
   int unsup = 0;
-  err = launch_ffn_stream(f, true, a1, p1, T, di.sms, di.smem_optin, st, &unsup);
+  err = launch_ffn_stream(f, true, a1, p1, T, di.sms, di.smem_optin, di.smem_per_sm, st, &unsup);
   if (unsup) return MOE_ERR_UNSUPPORTED;
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   if (q) {
@@ -211,7 +212,7 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
   a2.xexp = q ? hexp : nullptr;
   a2.out_routed = static_cast<__nv_bfloat16*>(y_perm);
   a2.out_shared = static_cast<__nv_bfloat16*>(y_shared);
-  err = launch_ffn_stream(f, false, a2, p2, T, di.sms, di.smem_optin, st, &unsup);
+  err = launch_ffn_stream(f, false, a2, p2, T, di.sms, di.smem_optin, di.smem_per_sm, st, &unsup);
   if (unsup) return MOE_ERR_UNSUPPORTED;
   return from_cuda(err);
 }
