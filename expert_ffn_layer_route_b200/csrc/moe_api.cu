@@ -11,10 +11,11 @@
 // Nothing here allocates device memory; all scratch is carved from the
 // caller's workspace.
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
-#include "ffn_stream.cuh"
+#include "ffn_gemm_tc.cuh"
 
 namespace moe {
 
@@ -190,6 +191,31 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
     a.K = (int)K;
     a.offsets = offsets;
   };
+  // Path: the tcgen05 grouped GEMM when experts average at least 64 rows
+  // (prefill-sized groups; bf16 weights), else the weight-streaming kernel.
+  // MOE_FFN_PATH=stream|gemm overrides the choice where both can run.
+  bool use_gemm = gemm_path_supported(f, F, D, true) && gemm_path_supported(f, D, F, false) &&
+                  (int64_t)T * k >= 64LL * E;
+  if (const char* e = getenv("MOE_FFN_PATH")) {
+    if (!strcmp(e, "stream")) use_gemm = false;
+    if (!strcmp(e, "gemm")) use_gemm = gemm_path_supported(f, F, D, true) && gemm_path_supported(f, D, F, false);
+  }
+  auto to_gemm = [&](const FfnArgs& s) {
+    GemmArgs g;
+    std::memset(&g, 0, sizeof(g));
+    g.offsets = s.offsets;
+    g.slot_map = s.slot_map;
+    g.n_phys = s.n_phys;
+    g.n_shared = s.n_shared;
+    g.E = s.E;
+    g.T = s.T;
+    g.k = s.k;
+    g.N = s.N;
+    g.K = s.K;
+    g.out_routed = s.out_routed;
+    g.out_shared = s.out_shared;
+    return g;
+  };
   FfnArgs a1;
   FfnPointers p1;
   fill(a1, p1, true);
@@ -198,7 +224,10 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
   a1.out_routed = h;
   a1.out_shared = nullptr;
   int unsup = 0;
-  err = launch_ffn_stream(f, true, a1, p1, T, di.sms, di.smem_optin, di.smem_per_sm, st, &unsup);
+  if (use_gemm)
+    err = launch_ffn_gemm(true, to_gemm(a1), p1, di.sms, di.smem_optin, st, &unsup);
+  else
+    err = launch_ffn_stream(f, true, a1, p1, T, di.sms, di.smem_optin, di.smem_per_sm, st, &unsup);
   if (unsup) return MOE_ERR_UNSUPPORTED;
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   if (q) {
@@ -212,7 +241,10 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
   a2.xexp = q ? hexp : nullptr;
   a2.out_routed = static_cast<__nv_bfloat16*>(y_perm);
   a2.out_shared = static_cast<__nv_bfloat16*>(y_shared);
-  err = launch_ffn_stream(f, false, a2, p2, T, di.sms, di.smem_optin, di.smem_per_sm, st, &unsup);
+  if (use_gemm)
+    err = launch_ffn_gemm(false, to_gemm(a2), p2, di.sms, di.smem_optin, st, &unsup);
+  else
+    err = launch_ffn_stream(f, false, a2, p2, T, di.sms, di.smem_optin, di.smem_per_sm, st, &unsup);
   if (unsup) return MOE_ERR_UNSUPPORTED;
   return from_cuda(err);
 }

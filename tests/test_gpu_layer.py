@@ -178,3 +178,39 @@ def test_full_size_layer_sampled_tokens(shape, T, tokens):
     H.check_permutation(res, shape)
     rel = H.check_output(res["out"], ref["out"], tokens=tokens)
     print(f"{shape.name} T={T}: rel err {rel:.2e} on {len(tokens)} tokens, ambiguous {n_amb}")
+
+
+# --------------------------------------------------- tensor-core GEMM path ----
+
+GEMM_CASES = [
+    ("bf16_gemm_ragged", mi.MIXTRAL.replace(d_model=512, d_ff=1024, n_experts=4), 300),
+    ("bf16_gemm_shared", mi.MIXTRAL.replace(d_model=512, d_ff=512, n_experts=8, n_shared=1), 200),
+    ("bf16_gemm_many_tiles", mi.MIXTRAL.replace(d_model=1024, d_ff=1536, n_experts=8), 1000),
+]
+
+
+@pytest.mark.parametrize("name,shape,T", GEMM_CASES, ids=[c[0] for c in GEMM_CASES])
+def test_gemm_path_matches_oracle_and_stream_path(name, shape, T, monkeypatch):
+    hl, dl = _layer(shape, T, 31)
+    monkeypatch.setenv("MOE_FFN_PATH", "gemm")
+    res = H.run_layer(dl)
+    rel, n_amb = H.full_check(hl, res)
+    monkeypatch.setenv("MOE_FFN_PATH", "stream")
+    res_s = H.run_layer(dl)
+    o1, o2 = res["out"].float(), res_s["out"].float()
+    # both are fp32-accumulated roundings of the same sums
+    assert (o1 - o2).abs().max().item() <= 1e-2 * o2.abs().max().item()
+    import expert_ffn_layer_route_b200 as moe
+    assert moe.moe_get_last_error() == 0
+    print(f"{name}: rel err {rel:.2e}, ambiguous {n_amb}")
+
+
+def test_gemm_path_full_size_prefill_sampled():
+    """Mixtral-shaped prefill (T=4096) through the default path (tensor-core GEMM)."""
+    hl, dl = _layer(mi.MIXTRAL, 4096, 12, device="cuda")
+    res = H.run_layer(dl)
+    tokens = [0, 1001, 2047, 4095]
+    ref, n_amb = H.check_routing(hl, res["idx"], res["gates"], tokens=tokens)
+    H.check_permutation(res, mi.MIXTRAL)
+    rel = H.check_output(res["out"], ref["out"], tokens=tokens)
+    print(f"mixtral T=4096: rel err {rel:.2e} on {len(tokens)} tokens, ambiguous {n_amb}")
