@@ -35,6 +35,8 @@ import moe_inputs as mi  # noqa: E402
 
 METRIC = "MoE-layer tokens/s and achieved HBM GB/s (decode) / TFLOPS (prefill) vs B200 peak"
 SHAPE = mi.GPTOSS
+DEFAULT_TOKENS = {"tiny": 16, "gptoss_decode": 64, "mixtral_prefill": 4096, "kimi_decode": 128,
+                  "offload_bank": 16}
 L2_BYTES = 126 * 2 ** 20
 
 
@@ -42,8 +44,9 @@ def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return {"hbm_gbs": d["hbm_gbs"], "src": "measured"}
-    return {"hbm_gbs": 6650.0, "src": "fallback"}
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
 
 
 def expert_bytes_split(shape):
@@ -183,7 +186,7 @@ def run_reference(args):
         return 0
     import torch
     from threadpoolctl import threadpool_limits
-    T = args.tokens
+    T = args.tokens or DEFAULT_TOKENS["gptoss_decode"]
     shape = SHAPE
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     budget = float(os.environ.get("MOE_REF_BUDGET_S", "150"))
@@ -226,20 +229,20 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------- our arm
-def kernel_src_sha():
-    p = os.path.join(ROOT, "expert_ffn_layer_route_b200", "csrc", "ffn_stream.cu")
+def kernel_src_sha(name="ffn_stream.cu"):
+    p = os.path.join(ROOT, "expert_ffn_layer_route_b200", "csrc", name)
     return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
 
 
-def stored_traffic(T):
+def stored_traffic(workload, T):
     """DRAM bytes per launch of the stage-1 kernel from a committed ncu summary,
     if it was taken on the current kernel source."""
     p = os.path.join(ROOT, "profiles", "ffn_stream_traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
-    ent = d.get(f"gptoss_decode_T{T}")
-    if not ent or ent.get("kernel_src_sha") != kernel_src_sha():
+    ent = d.get(f"{workload}_T{T}")
+    if not ent or ent.get("kernel_src_sha") != kernel_src_sha(ent.get("kernel_src_file", "ffn_stream.cu")):
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -259,17 +262,19 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
-    T = args.tokens
-    shape = SHAPE
+    shape = mi.CONFIGS[args.workload]
+    T = args.tokens or DEFAULT_TOKENS[args.workload]
     dlay = mi.draw_layer(shape, T, seed=1000 + rank, device=dev)
     desc = moe.make_desc(shape, T)
     ws = torch.empty(moe.moe_workspace_size(desc), dtype=torch.uint8, device=dev)
     out = torch.empty(T, shape.d_model, dtype=torch.bfloat16, device=dev)
     routed = moe.make_weights(dlay["experts"])
+    shared = moe.make_weights(dlay["shared"]) if dlay.get("shared") else None
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        moe.moe_layer_forward(desc, dlay["x"], dlay["router"], None, routed, None, out, ws, stream)
+    def step(x=None):
+        moe.moe_layer_forward(desc, dlay["x"] if x is None else x, dlay["router"], dlay["bias"], routed, shared,
+                              out, ws, stream)
 
     def barrier():
         if world > 1:
@@ -278,15 +283,21 @@ def run_ours(args):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
-    # routing of this batch -> algorithmic bytes
+    # routing of this batch -> algorithmic bytes / flops
     L = moe.moe_workspace_layout_of(desc)
     offs = ws[L.offsets: L.offsets + 4 * (shape.n_experts + 1)].view(torch.int32).cpu().numpy()
     distinct = int((np.diff(offs) > 0).sum())
     b13, b2 = expert_bytes_split(shape)
-    act_bytes = 2 * T * shape.d_model * 2
-    router_bytes = shape.n_experts * shape.d_model * 2
-    layer_bytes = distinct * (b13 + b2) + router_bytes + act_bytes
-    stage1_bytes = distinct * b13 + T * shape.d_model * 2 + T * shape.top_k * shape.d_ff * 2
+    d, f, k, S = shape.d_model, shape.d_ff, shape.top_k, shape.n_shared
+    act_bytes = 2 * T * d * 2
+    router_bytes = shape.n_experts * d * (4 if shape.router_fp32 else 2)
+    layer_bytes = (distinct + S) * (b13 + b2) + router_bytes + act_bytes
+    rows = T * k + S * T
+    layer_flops = 2.0 * rows * 3 * d * f + 2.0 * T * d * shape.n_experts
+    tensor_path = shape.wdtype == "bf16" and T * k >= 64 * shape.n_experts
+    kname = "ffn_gemm_stage1_gate_up" if tensor_path else "ffn_stage1_gate_up"
+    stage1_bytes = (distinct + S) * b13 + rows * d * 2 + rows * f * 2
+    stage1_flops = 2.0 * rows * d * 2 * f
 
     moe.moe_profile_enable(True)
     moe.moe_profile_collect()
@@ -320,12 +331,12 @@ def run_ours(args):
 
     # end to end: pinned host input -> device, layer, result -> pinned host, every step
     xh = dlay["x"].cpu().pin_memory()
-    oh = torch.empty(T, shape.d_model, dtype=torch.bfloat16).pin_memory()
+    oh = torch.empty(T, d, dtype=torch.bfloat16).pin_memory()
     xd = torch.empty_like(dlay["x"])
 
     def e2e_step():
         xd.copy_(xh, non_blocking=True)
-        moe.moe_layer_forward(desc, xd, dlay["router"], None, routed, None, out, ws, stream)
+        step(xd)
         oh.copy_(out, non_blocking=True)
 
     for _ in range(max(3, args.warmup)):
@@ -351,31 +362,42 @@ def run_ours(args):
 
     if rank == 0:
         pk = peaks()
-        s1 = prof.get("ffn_stage1_gate_up", (0, 0.0))
+        s1 = prof.get(kname, (0, 0.0))
         s1_ms = s1[1] / max(s1[0], 1)
-        achieved = stage1_bytes / (s1_ms * 1e-3) / 1e9 if s1_ms else 0.0
-        traffic = stored_traffic(T)
-        per_kernel = {k: {"launches": v[0], "avg_us": 1000.0 * v[1] / max(v[0], 1),
-                          "share": v[1] / max(sum(w[1] for w in prof.values()), 1e-12)} for k, v in prof.items()}
+        step_s = ms / args.steps * 1e-3
+        if tensor_path:
+            peak = pk["bf16_tflops_sustained"] if ms > 1000 else pk["bf16_tflops"]
+            achieved = stage1_flops / (s1_ms * 1e-3) / 1e12 if s1_ms else 0.0
+            roof = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": peak,
+                    "peak_source": pk["src"] + (" sustained" if ms > 1000 else " burst"), "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": stored_traffic(args.workload, T),
+                    "algorithmic_flops_per_launch": stage1_flops, "avg_launch_us": 1000 * s1_ms}
+        else:
+            achieved = stage1_bytes / (s1_ms * 1e-3) / 1e9 if s1_ms else 0.0
+            roof = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": pk["hbm_gbs"],
+                    "peak_source": pk["src"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                    "traffic": stored_traffic(args.workload, T),
+                    "algorithmic_bytes_per_launch": stage1_bytes, "avg_launch_us": 1000 * s1_ms}
+        per_kernel = {kk: {"launches": v[0], "avg_us": 1000.0 * v[1] / max(v[0], 1),
+                           "share": v[1] / max(sum(w[1] for w in prof.values()), 1e-12)} for kk, v in prof.items()}
         value = world * T * args.steps / (ms * 1e-3)
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": workload_name(shape, T), "tokens": T, "weights": "mxfp4",
-                       "parallelism": f"replicas x{world} (independent decode batches)",
-                       "l2": f"inputs larger than L2: {distinct} distinct experts = "
-                             f"{distinct * (b13 + b2) / 1e9:.2f} GB of weights per step vs {L2_BYTES / 2**20:.0f} MiB L2",
-                       "distinct_experts": distinct, "layer_algorithmic_bytes": layer_bytes,
-                       "layer_achieved_gbs": layer_bytes / (ms / args.steps * 1e-3) / 1e9},
-            "roofline": {"bound": "hbm", "kernel": "ffn_stage1_gate_up", "achieved": achieved,
-                         "peak": pk["hbm_gbs"], "peak_source": pk["src"], "unit": "GB/s",
-                         "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
-                         "algorithmic_bytes_per_launch": stage1_bytes, "avg_launch_us": 1000 * s1_ms},
+            "config": {"workload": workload_name(shape, T), "tokens": T, "weights": shape.wdtype,
+                       "parallelism": f"replicas x{world} (independent batches)",
+                       "l2": f"inputs larger than L2: {distinct + S} distinct experts = "
+                             f"{(distinct + S) * (b13 + b2) / 1e9:.2f} GB of weights per step vs "
+                             f"{L2_BYTES / 2**20:.0f} MiB L2",
+                       "distinct_experts": distinct + S, "layer_algorithmic_bytes": layer_bytes,
+                       "layer_achieved_gbs": layer_bytes / step_s / 1e9,
+                       "layer_algorithmic_flops": layer_flops, "layer_achieved_tflops": layer_flops / step_s / 1e12},
+            "roofline": roof,
             "kernels": per_kernel,
             "gpu_launches": launches,
             "e2e": {"value": world * T * args.steps / (ms_e2e * 1e-3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": T * shape.d_model * 2, "d2h_bytes_per_step": T * shape.d_model * 2},
+                    "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2},
             "clocks": clk,
             "cpu_baseline": cpu,
         }
@@ -391,7 +413,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--tokens", type=int, default=64)
+    ap.add_argument("--tokens", type=int, default=0, help="tokens per step (default: the workload's)")
+    ap.add_argument("--workload", choices=sorted(DEFAULT_TOKENS), default="gptoss_decode")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
