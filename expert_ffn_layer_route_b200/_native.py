@@ -258,12 +258,14 @@ class ExpertCache:
         _check(lib().moe_cache_prefetch(self.handle, layer, arr, n), "moe_cache_prefetch")
 
     def lookup(self, layer: int, experts, slot_map_dev, stream=None):
+        """slot_map_dev may be None for a policy-only cache (device < 0)."""
         arr, n = self._ints(experts)
-        _check(lib().moe_cache_lookup(self.handle, layer, arr, n, _ptr(slot_map_dev), _stream(stream)),
-               "moe_cache_lookup")
+        st = _stream(stream) if self.desc.device >= 0 else None
+        _check(lib().moe_cache_lookup(self.handle, layer, arr, n, _ptr(slot_map_dev), st), "moe_cache_lookup")
 
     def release(self, layer: int, stream=None):
-        _check(lib().moe_cache_release(self.handle, layer, _stream(stream)), "moe_cache_release")
+        st = _stream(stream) if self.desc.device >= 0 else None
+        _check(lib().moe_cache_release(self.handle, layer, st), "moe_cache_release")
 
     def slot_map(self, layer: int):
         out = (ctypes.c_int32 * self.n_experts)()

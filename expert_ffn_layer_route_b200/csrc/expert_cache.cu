@@ -50,6 +50,7 @@ struct moe_cache {
   std::vector<std::pair<cudaEvent_t, cudaEvent_t>> timing;  // pending copy timings
   std::vector<cudaEvent_t> free_events;
   bool inject_copy = false;
+  bool policy_only = false;  // device < 0: replacement policy and counters only, no CUDA calls
 };
 
 namespace {
@@ -151,11 +152,13 @@ moe_status place(moe_cache* c, int l, int e, const std::vector<int>& protect, Co
     pending(c, l, victim) = 0;
     c->st.evictions++;
   }
-  moe_status s = batch.begin(l);
-  if (s != MOE_OK) return s;
-  if (cudaMemcpyAsync(slot_ptr(c, l, slot), host_ptr(c, l, e), (size_t)c->d.expert_bytes, cudaMemcpyHostToDevice,
-                      c->copy_stream) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  if (!c->policy_only) {
+    moe_status s = batch.begin(l);
+    if (s != MOE_OK) return s;
+    if (cudaMemcpyAsync(slot_ptr(c, l, slot), host_ptr(c, l, e), (size_t)c->d.expert_bytes, cudaMemcpyHostToDevice,
+                        c->copy_stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   expert_in(c, l, slot) = e;
   slot_of(c, l, e) = slot;
   c->slot_seq[(size_t)l * C + slot] = ++c->copy_seq;
@@ -196,10 +199,24 @@ moe_status moe_cache_init(moe_cache** out, const moe_cache_desc* d) {
     return MOE_ERR_INVALID_ARG;
   const char* inj = std::getenv("MOE_FAULT_INJECT");
   const std::string inject = inj ? inj : "";
-  if (cudaSetDevice(d->device) != cudaSuccess) return MOE_ERR_CUDA;
   moe_cache* c = new moe_cache();
   c->d = *d;
   c->inject_copy = inject == "copy";
+  c->policy_only = d->device < 0;
+  if (c->policy_only) {
+    c->slot_of.assign((size_t)d->n_layers * d->n_experts, -1);
+    c->expert_in.assign((size_t)d->n_layers * d->slots_per_layer, -1);
+    c->last_use.assign((size_t)d->n_layers * d->n_experts, 0);
+    c->pending_prefetch.assign((size_t)d->n_layers * d->n_experts, 0);
+    c->slot_seq.assign((size_t)d->n_layers * d->slots_per_layer, 0);
+    c->released_valid.assign(d->n_layers, 0);
+    *out = c;
+    return MOE_OK;
+  }
+  if (cudaSetDevice(d->device) != cudaSuccess) {
+    delete c;
+    return MOE_ERR_CUDA;
+  }
   const size_t bank = (size_t)d->n_layers * d->n_experts * (size_t)d->expert_bytes;
   const size_t pool = (size_t)d->n_layers * d->slots_per_layer * (size_t)d->expert_bytes;
   moe_status st = MOE_OK;
@@ -242,12 +259,12 @@ moe_status moe_cache_init(moe_cache** out, const moe_cache_desc* d) {
 }
 
 void* moe_cache_host_expert(moe_cache* c, int32_t layer, int32_t e) {
-  if (!c || layer < 0 || layer >= c->d.n_layers || e < 0 || e >= c->d.n_experts) return nullptr;
+  if (!c || c->policy_only || layer < 0 || layer >= c->d.n_layers || e < 0 || e >= c->d.n_experts) return nullptr;
   return host_ptr(c, layer, e);
 }
 
 void* moe_cache_slot_base(moe_cache* c, int32_t layer) {
-  if (!c || layer < 0 || layer >= c->d.n_layers) return nullptr;
+  if (!c || c->policy_only || layer < 0 || layer >= c->d.n_layers) return nullptr;
   return slot_ptr(c, layer, 0);
 }
 
@@ -273,7 +290,8 @@ moe_status moe_cache_prefetch(moe_cache* c, int32_t layer, const int32_t* expert
 
 moe_status moe_cache_lookup(moe_cache* c, int32_t layer, const int32_t* experts, int32_t n, int32_t* slot_map_dev,
                             void* compute_stream) {
-  if (!c || layer < 0 || layer >= c->d.n_layers || !valid_list(c, experts, n) || !slot_map_dev)
+  if (!c || layer < 0 || layer >= c->d.n_layers || !valid_list(c, experts, n) ||
+      (!slot_map_dev && !c->policy_only))
     return MOE_ERR_INVALID_ARG;
   const std::vector<int> need = sorted_unique(experts, n);
   if (c->inject_copy && needs_copy(c, layer, need)) {
@@ -305,6 +323,7 @@ moe_status moe_cache_lookup(moe_cache* c, int32_t layer, const int32_t* experts,
   }
   moe_status s = batch.end();
   if (s != MOE_OK) return s;
+  if (c->policy_only) return MOE_OK;
   if (newest > c->waited_seq) {
     // copies are issued in order on one stream: waiting for the newest covers the rest
     if (cudaEventRecord(c->copy_done, c->copy_stream) != cudaSuccess) return MOE_ERR_CUDA;
@@ -323,6 +342,7 @@ moe_status moe_cache_lookup(moe_cache* c, int32_t layer, const int32_t* experts,
 
 moe_status moe_cache_release(moe_cache* c, int32_t layer, void* compute_stream) {
   if (!c || layer < 0 || layer >= c->d.n_layers) return MOE_ERR_INVALID_ARG;
+  if (c->policy_only) return MOE_OK;
   if (cudaEventRecord(c->released[layer], static_cast<cudaStream_t>(compute_stream)) != cudaSuccess)
     return MOE_ERR_CUDA;
   c->released_valid[layer] = 1;
@@ -337,13 +357,17 @@ moe_status moe_cache_slot_map(const moe_cache* c, int32_t layer, int32_t* out) {
 
 moe_status moe_cache_stats(moe_cache* c, moe_cache_stats_t* out) {
   if (!c || !out) return MOE_ERR_INVALID_ARG;
-  harvest_timing(c, true);
+  if (!c->policy_only) harvest_timing(c, true);
   *out = c->st;
   return MOE_OK;
 }
 
 moe_status moe_cache_destroy(moe_cache* c) {
   if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->policy_only) {
+    delete c;
+    return MOE_OK;
+  }
   if (c->copy_stream) cudaStreamSynchronize(c->copy_stream);
   for (auto& pr : c->timing) {
     cudaEventDestroy(pr.first);

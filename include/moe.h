@@ -216,7 +216,9 @@ typedef struct {
   int64_t expert_bytes;    /* bytes of one expert blob (multiple of 16) */
   void* host_bank;         /* host: pinned [n_layers][n_experts][expert_bytes], or NULL to
                               allocate (cudaHostAlloc) */
-  int32_t device;          /* CUDA device of the slots */
+  int32_t device;          /* CUDA device of the slots; < 0: policy only (no memory, no copies, no
+                              CUDA calls; lookup accepts a NULL slot map) - the replacement
+                              policy and counters alone, for replaying traces */
 } moe_cache_desc;
 
 typedef struct {
