@@ -228,6 +228,23 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------- multi-rank plumbing
+def max_over_ranks(value: float, world: int, device="cpu") -> float:
+    """The largest value over all ranks (timings are reported as the slowest rank's)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(world: int, tokens: int, steps: int, ms: float) -> float:
+    """All ranks' tokens (each rank runs its own batch) over the slowest rank's time."""
+    return world * tokens * steps / (ms * 1e-3)
+
+
 # ----------------------------------------------------------------- our arm
 def kernel_src_sha(name="ffn_stream.cu"):
     p = os.path.join(ROOT, "expert_ffn_layer_route_b200", "csrc", name)
@@ -322,11 +339,7 @@ def run_ours(args):
     clk = clocks.stop() if clocks else None
     moe.moe_profile_enable(False)
     prof = moe.moe_profile_collect()
-    ms = e0.elapsed_time(e1)
-    t_max = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    ms = float(t_max.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     launches = int(sum(v[0] for v in prof.values()))
 
     # end to end: pinned host input -> device, layer, result -> pinned host, every step
@@ -351,10 +364,7 @@ def run_ours(args):
     e3.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    ms_e2e = torch.tensor([e2.elapsed_time(e3)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms_e2e, op=dist.ReduceOp.MAX)
-    ms_e2e = float(ms_e2e.item())
+    ms_e2e = max_over_ranks(e2.elapsed_time(e3), world, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -380,7 +390,7 @@ def run_ours(args):
                     "algorithmic_bytes_per_launch": stage1_bytes, "avg_launch_us": 1000 * s1_ms}
         per_kernel = {kk: {"launches": v[0], "avg_us": 1000.0 * v[1] / max(v[0], 1),
                            "share": v[1] / max(sum(w[1] for w in prof.values()), 1e-12)} for kk, v in prof.items()}
-        value = world * T * args.steps / (ms * 1e-3)
+        value = whole_job_tokens_per_s(world, T, args.steps, ms)
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -396,7 +406,7 @@ def run_ours(args):
             "roofline": roof,
             "kernels": per_kernel,
             "gpu_launches": launches,
-            "e2e": {"value": world * T * args.steps / (ms_e2e * 1e-3), "unit": "tokens/s",
+            "e2e": {"value": whole_job_tokens_per_s(world, T, args.steps, ms_e2e), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2},
             "clocks": clk,
             "cpu_baseline": cpu,

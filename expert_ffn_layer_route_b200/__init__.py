@@ -34,4 +34,5 @@ from ._native import (  # noqa: F401
     router_sum_depth,
     moe_profile_enable,
     moe_profile_collect,
+    moe_diag_wait_timeout,
 )

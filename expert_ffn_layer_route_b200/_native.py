@@ -82,6 +82,7 @@ _SIGS = {
     "moe_cache_destroy": [_P],
     "moe_get_last_error": [],
     "moe_profile_enable": [ctypes.c_int],
+    "moe_diag_wait_timeout": [ctypes.c_uint64, _P, _P],
     "moe_profile_collect": [ctypes.POINTER(ProfileEntry), ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)],
 }
 _PTR_RET = {"moe_cache_host_expert": [_P, ctypes.c_int32, ctypes.c_int32],
@@ -216,6 +217,10 @@ def moe_layer_forward(desc, x, w_router, logit_bias, routed: Weights, shared: Op
 
 def moe_get_last_error() -> int:
     return lib().moe_get_last_error()
+
+
+def moe_diag_wait_timeout(limit_ns: int, finished, stream=None):
+    _check(lib().moe_diag_wait_timeout(int(limit_ns), _ptr(finished), _stream(stream)), "moe_diag_wait_timeout")
 
 
 def moe_profile_enable(on: bool = True):

@@ -386,3 +386,29 @@ moe_status moe_get_last_error(void) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Diagnostic: the bounded wait every pipelined kernel uses, made to run out.
+// One CTA waits on an mbarrier phase that nothing completes, with the given
+// limit; the wait gives up, records MOE_ERR_TIMEOUT in the status word and
+// the kernel returns normally, so the context stays usable.
+namespace moe {
+__global__ void wait_timeout_probe_kernel(uint64_t limit_ns, int* finished) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = mbar_wait_limit(&bar, 0, limit_ns);  // phase 0 never completes
+    *finished = ok ? 2 : 1;
+  }
+}
+}  // namespace moe
+
+extern "C" moe_status moe_diag_wait_timeout(uint64_t limit_ns, int32_t* finished, void* stream) {
+  if (!finished || limit_ns > 10000000000ull) return MOE_ERR_INVALID_ARG;
+  moe::wait_timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, finished);
+  return from_cuda(cudaGetLastError());
+}

@@ -265,6 +265,14 @@ typedef struct {
 moe_status moe_profile_enable(int on);
 moe_status moe_profile_collect(moe_profile_entry* out, int32_t cap, int32_t* n_out);
 
+/* Diagnostic, no counterpart in the pages: launches one CTA that waits, with
+ * the bounded wait every pipelined kernel here uses, on an mbarrier phase that
+ * nothing completes.  After `limit_ns` (<= 10 s) the wait gives up, records
+ * MOE_ERR_TIMEOUT in the device status word, writes 1 to *finished (device
+ * int32) and the kernel returns: the failure path of a stuck pipeline,
+ * exercised without hanging or faulting the GPU. */
+moe_status moe_diag_wait_timeout(uint64_t limit_ns, int32_t* finished, void* stream);
+
 const char* moe_status_string(moe_status s);
 /* Synchronises the current device, returns and clears the device status word. */
 moe_status moe_get_last_error(void);

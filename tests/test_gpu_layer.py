@@ -214,3 +214,19 @@ def test_gemm_path_full_size_prefill_sampled():
     H.check_permutation(res, mi.MIXTRAL)
     rel = H.check_output(res["out"], ref["out"], tokens=tokens)
     print(f"mixtral T=4096: rel err {rel:.2e} on {len(tokens)} tokens, ambiguous {n_amb}")
+
+
+def test_bounded_wait_times_out_with_status_and_context_survives():
+    """A pipeline wait that can never be satisfied gives up after its limit,
+    reports MOE_ERR_TIMEOUT, and the GPU keeps working afterwards."""
+    import time
+    import expert_ffn_layer_route_b200 as moe
+    moe.moe_get_last_error()
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0 = time.perf_counter()
+    moe.moe_diag_wait_timeout(50_000_000, flag)  # 50 ms
+    assert moe.moe_get_last_error() == 6  # MOE_ERR_TIMEOUT (synchronises)
+    assert time.perf_counter() - t0 < 5.0
+    assert flag.item() == 1
+    hl, dl = _layer(mi.TINY, 16, 0)
+    H.full_check(hl, H.run_layer(dl))  # the context is still usable
