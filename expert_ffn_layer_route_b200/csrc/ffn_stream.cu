@@ -66,6 +66,11 @@ struct FmtTraits<kINT4> {
 
 __device__ __forceinline__ int sigma8(int g) { return (g >> 1) | ((g & 1) << 2); }
 
+// Shared-memory header: barriers, flags, offsets [E+1], group table.
+__host__ __device__ constexpr int stream_hdr_bytes(int E, int n_shared) {
+  return ((16 * kMaxStages + 64 + 4 * ((E + 4) + 2 * (E + n_shared + 4))) + 1023) & ~1023;
+}
+
 // Everything a block needs to know about one work item.
 struct Item {
   int valid;
@@ -74,18 +79,33 @@ struct Item {
   int xrow0;       // first activation / output row of this expert
   int n_cols;      // activation rows of this expert
   int phys;        // physical expert index (TMA coordinate)
+  int pass;        // which XCOLS-wide slice of the expert's rows
   const uint8_t* sbase;
   float gscale;
 };
 
+// Work items are (group, tile, pass): groups are the shared experts then the
+// routed experts with rows (gitem holds each group's first item), and every
+// pass of XCOLS activation rows is its own item, passes fastest, so that the
+// CTAs streaming one weight tile for different passes run side by side and
+// share it through L2.
 template <int F>
-__device__ __forceinline__ Item decode_item(const FfnArgs& a, int item, int ntile, const int* act,
-                                            const int* offs) {
+__device__ __forceinline__ Item decode_item(const FfnArgs& a, int item, int ntile, const int* gitem,
+                                            const int* gexp, int ngroups, const int* offs) {
   Item it{};
-  const int grp = item / ntile;
-  it.tile = item - grp * ntile;
+  int lo = 0, hi = ngroups - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (gitem[mid] <= item) lo = mid; else hi = mid - 1;
+  }
+  const int passes = (gitem[lo + 1] - gitem[lo]) / ntile;
+  const int local = item - gitem[lo];
+  it.tile = local / passes;
+  it.pass = local - it.tile * passes;
   it.valid = 1;
-  if (grp < a.n_shared) {
+  const int ex = gexp[lo];
+  const int grp = ex < 0 ? -1 - ex : a.n_shared + ex;
+  if (ex < 0) {
     it.shared_idx = grp;
     it.xrow0 = a.T * a.k + grp * a.T;
     it.n_cols = a.T;
@@ -93,7 +113,7 @@ __device__ __forceinline__ Item decode_item(const FfnArgs& a, int item, int ntil
     it.sbase = a.s_sh ? a.s_sh + (int64_t)grp * a.stride_s_sh : nullptr;
     it.gscale = (F == kNVFP4 && a.gsc_sh) ? __ldg(a.gsc_sh + grp) : 1.f;
   } else {
-    const int e = act[grp - a.n_shared];
+    const int e = ex;
     it.shared_idx = -1;
     it.xrow0 = offs[e];
     it.n_cols = offs[e + 1] - offs[e];
@@ -133,10 +153,11 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
   uint64_t* sfull = empty + kMaxStages;
   uint64_t* sempty = sfull + 2;
   volatile int* s_abort = reinterpret_cast<volatile int*>(sempty + 2);
-  int* s_nact = reinterpret_cast<int*>(sempty + 2) + 1;
+  int* s_ngroups = reinterpret_cast<int*>(sempty + 2) + 1;
   int* s_offs = reinterpret_cast<int*>(sempty + 2) + 4;  // [E+1]
-  int* s_act = s_offs + (a.E + 4);                       // [E]
-  const int hdr = ((16 * kMaxStages + 32 + 16 + 8 * a.E + 64) + 1023) & ~1023;
+  int* s_gitem = s_offs + (a.E + 4);                     // [groups+1]
+  int* s_gexp = s_gitem + (a.E + a.n_shared + 4);        // [groups]
+  const int hdr = stream_hdr_bytes(a.E, a.n_shared);
   uint8_t* s_scale = smem + hdr;
   uint8_t* s_stage = s_scale + a.n_scale_buf * a.smem_scale_bytes;
 
@@ -155,23 +176,54 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
   }
   for (int i = tid; i <= E; i += kThreads) s_offs[i] = __ldg(a.offsets + i);
   __syncthreads();
-  if (warp == 0) {
-    int n = 0;
-    for (int base = 0; base < E; base += 32) {
-      const int e = base + lane;
-      const bool on = e < E && s_offs[e + 1] > s_offs[e];
-      const uint32_t m = __ballot_sync(0xffffffffu, on);
-      if (on) s_act[n + __popc(m & ((1u << lane) - 1u))] = e;
-      n += __popc(m);
-    }
-    if (lane == 0) *s_nact = n;
-  }
-  __syncthreads();
-  const int n_act = *s_nact;
-
   const int rows_per_item = kGateUp ? kRowsPerStage / 2 : kRowsPerStage;
   const int ntile = ceil_div(a.N, rows_per_item);
-  const int n_items = (a.n_shared + n_act) * ntile;
+  if (warp == 0) {
+    int ng = 0, items = 0;
+    for (int sh = 0; sh < a.n_shared; ++sh) {
+      if (lane == 0) {
+        s_gitem[ng] = items;
+        s_gexp[ng] = -1 - sh;
+      }
+      ++ng;
+      items += ntile * ceil_div(a.T, XCOLS);
+    }
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      int cnt_items = 0;
+      if (e < E) {
+        const int r0e = s_offs[e], cnt = s_offs[e + 1] - r0e;
+        const int p = a.slot_map ? __ldg(a.slot_map + e) : e;
+        bool ok = cnt > 0;
+        if (ok && (p < 0 || p >= a.n_phys || r0e < 0 || r0e + cnt > a.T * a.k)) {
+          if (!(p == -1 && a.slot_map)) set_status(MOE_ERR_DEVICE_INDEX);  // -1: not resident, skipped
+          ok = false;
+        }
+        cnt_items = ok ? ntile * ceil_div(cnt, XCOLS) : 0;
+      }
+      const uint32_t on = __ballot_sync(0xffffffffu, cnt_items > 0);
+      int incl = cnt_items;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      if (cnt_items > 0) {
+        const int slot = ng + __popc(on & ((1u << lane) - 1u));
+        s_gitem[slot] = items + incl - cnt_items;
+        s_gexp[slot] = e;
+      }
+      ng += __popc(on);
+      items += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      s_gitem[ng] = items;
+      *s_ngroups = ng;
+    }
+  }
+  __syncthreads();
+  const int ngroups = *s_ngroups;
+  const int n_items = s_gitem[ngroups];
   const int K = a.K;
   const int srow = Tr::blk ? (K / Tr::blk) * Tr::sbytes : 0;
   const int nchunks = ceil_div(K, KC);
@@ -185,25 +237,24 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
       prefetch_tmap(&a.tm_w);
       prefetch_tmap(&a.tm_x);
       if (a.n_shared) prefetch_tmap(&a.tm_wsh);
-      const uint64_t pol_w = l2_evict_first_policy();
+      const uint64_t pol_w = a.w_l2_normal ? l2_evict_normal_policy() : l2_evict_first_policy();
       const uint64_t pol_x = l2_evict_last_policy();
       uint32_t cnt = 0;
       int item_no = 0;
       for (int item = blockIdx.x; item < n_items && !*s_abort; item += gridDim.x, ++item_no) {
-        const Item it = decode_item<F>(a, item, ntile, s_act, s_offs);
+        const Item it = decode_item<F>(a, item, ntile, s_gitem, s_gexp, ngroups, s_offs);
         const int r0 = it.tile * rows_per_item;
         const int nrows = min(rows_per_item, a.N - r0);
-        const int passes = it.valid ? ceil_div(it.n_cols, XCOLS) : 0;
         const int sb = item_no % nsb;
         const uint32_t suse = item_no / nsb;
         const int sc_at = (nsb == 2) ? 0 : min(nstage - 1, nchunks - 1);
         const CUtensorMap* tw = it.shared_idx >= 0 ? &a.tm_wsh : &a.tm_w;
         // boxes of weight rows: stage 1 gate rows r0.. and up rows N+r0..; stage 2 rows r0.., r0+128..
         const int nbox_w = kGateUp ? 2 : (nrows > kBoxRows ? 2 : 1);
-        for (int pass = 0; pass < max(passes, 1) && !*s_abort; ++pass) {
+        for (int pass = it.pass; pass == it.pass && !*s_abort; ++pass) {
           const int c0 = pass * XCOLS;
           for (int ch = 0; ch < nchunks; ++ch) {
-            if (Tr::blk && pass == 0 && ch == sc_at) {
+            if (Tr::blk && ch == sc_at) {
               if (!mbar_wait(&sempty[sb], (suse & 1u) ^ 1u)) {
                 *s_abort = 1;
                 break;
@@ -261,10 +312,9 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
   const uint32_t stage0 = smem_u32(s_stage);
   const uint32_t scale0 = smem_u32(s_scale);
   for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++item_no) {
-    const Item it = decode_item<F>(a, item, ntile, s_act, s_offs);
+    const Item it = decode_item<F>(a, item, ntile, s_gitem, s_gexp, ngroups, s_offs);
     const int r0 = it.tile * rows_per_item;
     const int nrows = min(rows_per_item, a.N - r0);
-    const int passes = it.valid ? ceil_div(it.n_cols, XCOLS) : 0;
     const int sb = item_no % nsb;
     const uint32_t suse = item_no / nsb;
     // smem rows of this warp's two m16 tiles
@@ -275,9 +325,9 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
       if (!mbar_wait(&sfull[sb], suse & 1u)) *s_abort = 1;
     }
     const uint32_t sc_base = scale0 + sb * a.smem_scale_bytes;
-    for (int pass = 0; pass < max(passes, 1); ++pass) {
+    for (int pass = it.pass; pass == it.pass; ++pass) {
       const int c0 = pass * XCOLS;
-      const int ncols = passes ? min(XCOLS, it.n_cols - c0) : 0;
+      const int ncols = min(XCOLS, it.n_cols - c0);
       const int ng_act = ceil_div(ncols, 8);
       float acc[NG][2][4];
 #pragma unroll
@@ -512,8 +562,8 @@ static int fmt_srow(int F, int K) {
 }
 
 // Shared memory plan of one stage kernel; returns false when it cannot fit.
-static bool plan_smem(int F, int ng, int K, int E, int smem_max, FfnArgs& a, size_t& total) {
-  const int hdr = ((16 * kMaxStages + 32 + 16 + 8 * E + 64) + 1023) & ~1023;
+static bool plan_smem(int F, int ng, int K, int E, int n_shared, int smem_max, FfnArgs& a, size_t& total) {
+  const int hdr = stream_hdr_bytes(E, n_shared);
   const int sbuf = ((kRowsPerStage * fmt_srow(F, K)) + 1023) & ~1023;
   const int stage = kRowsPerStage * kLine + ((fmt_kc(F) * 2) / kLine) * ng * 8 * kLine;
   const int usable = smem_max - 1024;  // room for the runtime 1024-byte alignment
@@ -546,13 +596,14 @@ cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers&
   if (const char* e = getenv("MOE_FFN_NG")) ng = atoi(e);
   if (const char* e = getenv("MOE_FFN_MINB")) minb = atoi(e);
   if (ng != 1 && ng != 2 && ng != 4) ng = 2;
+  if (const char* e = getenv("MOE_W_L2NORMAL")) a.w_l2_normal = atoi(e);
   if (minb == 2 && ng > 2) ng = 2;
   size_t smem = 0;
   bool ok = false;
-  if (minb == 2) ok = plan_smem(F, ng, a.K, a.E, smem_per_sm / 2 - 1024, a, smem);
+  if (minb == 2) ok = plan_smem(F, ng, a.K, a.E, a.n_shared, smem_per_sm / 2 - 1024, a, smem);
   if (!ok) {
     minb = 1;
-    ok = plan_smem(F, ng, a.K, a.E, smem_max, a, smem);
+    ok = plan_smem(F, ng, a.K, a.E, a.n_shared, smem_max, a, smem);
   }
   if (!ok) {
     *unsupported = 1;

@@ -37,6 +37,7 @@ struct alignas(64) FfnArgs {
   int n_stages;
   int n_scale_buf;
   int smem_scale_bytes;  // per buffer
+  int w_l2_normal;       // 1: weight boxes with normal L2 priority, 0: evict-first
 };
 
 // Launch one stage (gate_up: stage 1 with SwiGLU; else stage 2) of the
