@@ -35,6 +35,7 @@ import moe_inputs as mi  # noqa: E402
 
 METRIC = "MoE-layer tokens/s and achieved HBM GB/s (decode) / TFLOPS (prefill) vs B200 peak"
 SHAPE = mi.GPTOSS
+PROFILE_EVERY = 10
 DEFAULT_TOKENS = {"tiny": 16, "gptoss_decode": 64, "mixtral_prefill": 4096, "kimi_decode": 128,
                   "offload_bank": 16}
 L2_BYTES = 126 * 2 ** 20
@@ -264,6 +265,14 @@ def stored_traffic(workload, T):
     return ent.get("dram_bytes_per_launch")
 
 
+def launches_per_step(prof, steps):
+    """Kernel launches in the timed region: the sampled steps' launch count per
+    step times the number of steps."""
+    sampled = (steps + PROFILE_EVERY - 1) // PROFILE_EVERY
+    per_step = sum(v[0] for v in prof.values()) / max(sampled, 1)
+    return int(round(per_step * steps))
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -316,7 +325,7 @@ def run_ours(args):
     stage1_bytes = (distinct + S) * b13 + rows * d * 2 + rows * f * 2
     stage1_flops = 2.0 * rows * d * 2 * f
 
-    moe.moe_profile_enable(True)
+    moe.moe_profile_enable(not args.no_kernel_timing)
     moe.moe_profile_collect()
     bus = -1
     try:
@@ -330,8 +339,13 @@ def run_ours(args):
     barrier()
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # per-kernel CUDA events on every PROFILE_EVERY-th step of the timed region
+    # (events between launches also stop a kernel from overlapping its
+    # predecessor, so they are sampled rather than put around every launch)
     e0.record(stream)
-    for _ in range(args.steps):
+    for i in range(args.steps):
+        if not args.no_kernel_timing:
+            moe.moe_profile_enable(i % PROFILE_EVERY == 0)
         step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
@@ -339,8 +353,8 @@ def run_ours(args):
     clk = clocks.stop() if clocks else None
     moe.moe_profile_enable(False)
     prof = moe.moe_profile_collect()
+    launches = launches_per_step(prof, args.steps)
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    launches = int(sum(v[0] for v in prof.values()))
 
     # end to end: pinned host input -> device, layer, result -> pinned host, every step
     xh = dlay["x"].cpu().pin_memory()
@@ -495,6 +509,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--bank-layers", type=int, default=8, help="layers of the offloaded bank (of 48)")
+    ap.add_argument("--no-kernel-timing", action="store_true",
+                    help="no per-kernel CUDA events in the timed region (the roofline fields are then empty)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -255,3 +255,14 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __int_as_
 __host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 }  // namespace moe
+
+namespace moe {
+// Programmatic dependent launch: every kernel of the library waits for the
+// previous kernel in its stream (griddepcontrol.wait) before its first global
+// memory access, then lets the next kernel start launching.  Launched without
+// the PDL attribute, both instructions are no-ops.
+__device__ __forceinline__ void pdl_wait_and_trigger() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+}  // namespace moe

@@ -29,6 +29,7 @@
 #include <cstdlib>
 
 #include "ffn_gemm_tc.cuh"
+#include "launch.cuh"
 #include "profile.cuh"
 #include "tc_ptx.cuh"
 
@@ -93,6 +94,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ffn_gemm_tc_kernel(const __grid
     *s_abort = 0;
     fence_barrier_init();
   }
+  pdl_wait_and_trigger();
   // Group table: shared experts first, then routed experts with rows, each
   // with its number of 128-row m-tiles (non-resident experts get none).
   if (warp == 0) {
@@ -349,8 +351,7 @@ static cudaError_t launch_gemm(const GemmArgs& a, int grid, size_t smem, cudaStr
     configured = (int)smem;
   }
   ProfScope prof(GU ? "ffn_gemm_stage1_gate_up" : "ffn_gemm_stage2_down", st);
-  kern<<<grid, kThreadsTc, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreadsTc), smem, st, a);
 }
 
 cudaError_t launch_ffn_gemm(bool gate_up, GemmArgs a, const GemmPointers& p, int n_sms, int smem_max,

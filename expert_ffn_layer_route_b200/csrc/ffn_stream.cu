@@ -32,6 +32,7 @@
 #include <cstdlib>
 
 #include "ffn_stream.cuh"
+#include "launch.cuh"
 #include "profile.cuh"
 
 namespace moe {
@@ -174,6 +175,7 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
     *s_abort = 0;
     fence_barrier_init();
   }
+  pdl_wait_and_trigger();
   for (int i = tid; i <= E; i += kThreads) s_offs[i] = __ldg(a.offsets + i);
   __syncthreads();
   const int rows_per_item = kGateUp ? kRowsPerStage / 2 : kRowsPerStage;
@@ -532,8 +534,7 @@ static cudaError_t launch_one(const FfnArgs& a, int grid, size_t smem, cudaStrea
     configured_smem = (int)smem;
   }
   ProfScope prof(GU ? "ffn_stage1_gate_up" : "ffn_stage2_down", st);
-  kern<<<grid, kThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, a);
 }
 
 template <int F, bool GU>

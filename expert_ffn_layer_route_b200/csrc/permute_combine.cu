@@ -16,6 +16,7 @@
 // the 128 routed experts": "Mixture of experts VRAM: total vs active
 // parameters", section "How current MoE models route each token").
 #include "common.cuh"
+#include "launch.cuh"
 #include "profile.cuh"
 
 namespace moe {
@@ -32,6 +33,7 @@ __global__ void __launch_bounds__(kPermThreads)
   int* tile = sm + 2 * E;      // [kPermTile]
   __shared__ int wsum[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait_and_trigger();
   for (int e = tid; e < E; e += kPermThreads) counts[e] = 0;
   __syncthreads();
   for (int i = tid; i < n; i += kPermThreads) {
@@ -101,8 +103,8 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* off
   cudaError_t err = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   ProfScope prof("permute", st);
-  permute_kernel<<<1, kPermThreads, smem, st>>>(idx, T * k, k, E, offsets, row_token, inv);
-  return cudaGetLastError();
+  return launch_pdl(permute_kernel, dim3(1), dim3(kPermThreads), smem, st, idx, T * k, k, E, offsets, row_token,
+                    inv);
 }
 
 // ---------------------------------------------------------------------------
@@ -122,6 +124,7 @@ template <int kMode>
 __global__ void __launch_bounds__(kPrepThreads)
     prep_rows_kernel(const __nv_bfloat16* __restrict__ src, int K, void* __restrict__ dst,
                      int32_t* __restrict__ rexp, const int32_t* __restrict__ gather, int n_gather, int n_tok) {
+  pdl_wait_and_trigger();
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
   int srow = row;
@@ -189,12 +192,13 @@ cudaError_t launch_prep_rows(const void* src, int rows, int K, int mode, void* d
   ProfScope prof(gather ? "prep_x_gather" : "prep_h", st);
   const __nv_bfloat16* s = static_cast<const __nv_bfloat16*>(src);
   if (mode == kCopyBf16)
-    prep_rows_kernel<kCopyBf16><<<rows, kPrepThreads, 0, st>>>(s, K, dst, rexp, gather, n_gather, n_tok);
-  else if (mode == kF16PermInt4)
-    prep_rows_kernel<kF16PermInt4><<<rows, kPrepThreads, 0, st>>>(s, K, dst, rexp, gather, n_gather, n_tok);
-  else
-    prep_rows_kernel<kF16><<<rows, kPrepThreads, 0, st>>>(s, K, dst, rexp, gather, n_gather, n_tok);
-  return cudaGetLastError();
+    return launch_pdl(prep_rows_kernel<kCopyBf16>, dim3(rows), dim3(kPrepThreads), 0, st, s, K, dst, rexp, gather,
+                      n_gather, n_tok);
+  if (mode == kF16PermInt4)
+    return launch_pdl(prep_rows_kernel<kF16PermInt4>, dim3(rows), dim3(kPrepThreads), 0, st, s, K, dst, rexp,
+                      gather, n_gather, n_tok);
+  return launch_pdl(prep_rows_kernel<kF16>, dim3(rows), dim3(kPrepThreads), 0, st, s, K, dst, rexp, gather,
+                    n_gather, n_tok);
 }
 
 // ---------------------------------------------------------------------------
@@ -204,6 +208,7 @@ __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const __nv_bfloat16* __restrict__ y, const int32_t* __restrict__ inv,
                    const float* __restrict__ gw, const __nv_bfloat16* __restrict__ y_shared, int n_shared, int T,
                    int d, int k, __nv_bfloat16* __restrict__ out) {
+  pdl_wait_and_trigger();
   const int t = blockIdx.x;
   const int nchunk = d / 8;
   const int nrows = T * k;
@@ -246,10 +251,9 @@ cudaError_t launch_combine(const void* y, const int32_t* inv, const float* gw, c
                            int T, int d, int k, void* out, cudaStream_t st) {
   if (T <= 0) return cudaSuccess;
   ProfScope prof("combine", st);
-  combine_kernel<<<T, kCombineThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(y), inv, gw,
-                                                static_cast<const __nv_bfloat16*>(y_shared), n_shared, T, d, k,
-                                                static_cast<__nv_bfloat16*>(out));
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(T), dim3(kCombineThreads), 0, st, static_cast<const __nv_bfloat16*>(y), inv,
+                    gw, static_cast<const __nv_bfloat16*>(y_shared), n_shared, T, d, k,
+                    static_cast<__nv_bfloat16*>(out));
 }
 
 }  // namespace moe

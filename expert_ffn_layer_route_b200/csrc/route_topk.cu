@@ -21,6 +21,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "launch.cuh"
 #include "profile.cuh"
 
 namespace moe {
@@ -33,6 +34,7 @@ template <bool kFp32Router>
 __global__ void __launch_bounds__(kRouterThreads)
     router_logits_kernel(const __nv_bfloat16* __restrict__ x, const void* __restrict__ wr,
                          const float* __restrict__ bias, float* __restrict__ logits, int T, int d, int E) {
+  pdl_wait_and_trigger();
   const int t0 = blockIdx.x * kRouterTokens;
   const int e0 = blockIdx.y * kRouterExperts;
   const int tid = threadIdx.x;
@@ -120,6 +122,7 @@ __device__ __forceinline__ bool beats(float v, int i, float w, int j) {
 __global__ void __launch_bounds__(256)
     topk_kernel(const float* __restrict__ logits, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                 int T, int E, int k) {
+  pdl_wait_and_trigger();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= T) return;
@@ -169,18 +172,19 @@ cudaError_t launch_route_topk(const moe_layer_desc& dsc, const void* x, const vo
   dim3 grid(ceil_div(T, kRouterTokens), ceil_div(E, kRouterExperts));
   {
   ProfScope prof("router_logits", st);
+  cudaError_t err;
   if (dsc.router_fp32)
-    router_logits_kernel<true><<<grid, kRouterThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x), wr, bias,
-                                                                  logits, T, d, E);
+    err = launch_pdl(router_logits_kernel<true>, grid, dim3(kRouterThreads), 0, st,
+                     static_cast<const __nv_bfloat16*>(x), wr, bias, logits, T, d, E);
   else
-    router_logits_kernel<false><<<grid, kRouterThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x), wr, bias,
-                                                                   logits, T, d, E);
+    err = launch_pdl(router_logits_kernel<false>, grid, dim3(kRouterThreads), 0, st,
+                     static_cast<const __nv_bfloat16*>(x), wr, bias, logits, T, d, E);
+  if (err != cudaSuccess) return err;
   }
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   ProfScope prof("topk", st);
-  topk_kernel<<<ceil_div(T * 32, 256), 256, 0, st>>>(logits, topk_idx, topk_w, T, E, k);
-  return cudaGetLastError();
+  return launch_pdl(topk_kernel, dim3(ceil_div(T * 32, 256)), dim3(256), 0, st, logits, topk_idx, topk_w, T, E, k);
 }
 
 }  // namespace moe
