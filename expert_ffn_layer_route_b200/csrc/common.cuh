@@ -185,6 +185,15 @@ __device__ __forceinline__ void e8m0x2_to_f32x2(uint32_t pair16, float& lo, floa
   hi = __uint_as_float(b2 & 0xffff0000u);
 }
 
+// (d0, d1) += (a0, a1) * s with one packed fp32x2 FMA (each lane rounds once,
+// exactly like two fmaf).
+__device__ __forceinline__ void ffma2_scalar(float& d0, float& d1, float a0, float a1, float s) {
+  asm("{\n .reg .b64 rd, ra, rs;\n mov.b64 ra, {%2, %3};\n mov.b64 rs, {%4, %4};\n mov.b64 rd, {%0, %1};\n"
+      " fma.rn.f32x2 rd, ra, rs, rd;\n mov.b64 {%0, %1}, rd;\n}\n"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1), "f"(s));
+}
+
 // D = A * B (accumulator starts at zero).
 __device__ __forceinline__ void mma_f16_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {

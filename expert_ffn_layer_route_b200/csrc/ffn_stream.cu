@@ -349,28 +349,36 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
           const uint32_t wst = stage0 + s * STAGE_BYTES;
           const uint32_t xst = wst + W_BYTES;
           const int nblk = min(KC, K - ch * KC) / 32;
-          // 32-wide K blocks in pairs: the MXFP4 scales of a pair load as one
-          // 16-bit value per row (low byte: even block)
-          const bool pair_aligned = (srow & 1) == 0;
-          for (int bp = 0; bp < nblk; bp += 2) {
-            float scp[2][2][2];  // MXFP4 scales [m-tile][row g / g+8][block of the pair]
-            if constexpr (F == kMXFP4) {
-              const int blk = (ch * KC) / 32 + bp;
+          // MXFP4 block scales of this chunk: the four lanes of a quad need the
+          // same four rows, so lane c converts the chunk's eight scales of one
+          // of them (m-tile c>>1, row g + 8(c&1)), two per 16-bit load, and the
+          // quad shares them through shuffles.
+          float sc8[KC / 32];
+          if constexpr (F == kMXFP4) {
+            const bool pair_aligned = (srow & 1) == 0;
+            const uint32_t ad0 = sc_base + (((c >> 1) ? m1 : m0) + g + 8 * (c & 1)) * srow + (ch * KC) / 32;
 #pragma unroll
-              for (int mt = 0; mt < 2; ++mt) {
-                const int mr = mt ? m1 : m0;
-#pragma unroll
-                for (int hr = 0; hr < 2; ++hr) {
-                  const uint32_t ad = sc_base + (mr + g + 8 * hr) * srow + blk;
-                  const uint32_t v = pair_aligned ? lds16(ad) : (lds8(ad) | (lds8(ad + 1) << 8));
-                  e8m0x2_to_f32x2(v, scp[mt][hr][0], scp[mt][hr][1]);
-                }
-              }
+            for (int p = 0; p < KC / 64; ++p) {
+              uint32_t v = 0x7f7fu;  // past the row's last block: unused
+              if (2 * p < nblk) v = pair_aligned ? lds16(ad0 + 2 * p) : (lds8(ad0 + 2 * p) | (lds8(ad0 + 2 * p + 1) << 8));
+              e8m0x2_to_f32x2(v, sc8[2 * p], sc8[2 * p + 1]);
             }
+          }
+#pragma unroll
+          for (int bp = 0; bp < KC / 32; bp += 2) {
+            if (bp >= nblk) break;
 #pragma unroll
             for (int hb = 0; hb < 2; ++hb) {
             const int b = bp + hb;
             if (b >= nblk) break;
+            float scb[2][2];  // MXFP4 scale of block b for [m-tile][row g / g+8]
+            if constexpr (F == kMXFP4) {
+#pragma unroll
+              for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr)
+                  scb[mt][hr] = __shfl_sync(0xffffffffu, sc8[b], (lane & ~3) | (2 * mt + hr));
+            }
             uint32_t A[2][2][4];  // [m-tile][k16 tile][reg]
             if constexpr (F == kBF16) {
 #pragma unroll
@@ -433,10 +441,8 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
                     float t4[4];
                     mma_f16_z(t4, A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
                     mma_f16(t4, A[mt][1][0], A[mt][1][1], A[mt][1][2], A[mt][1][3], xv.z, xv.w);
-                    acc[q][mt][0] = fmaf(t4[0], scp[mt][0][hb], acc[q][mt][0]);
-                    acc[q][mt][1] = fmaf(t4[1], scp[mt][0][hb], acc[q][mt][1]);
-                    acc[q][mt][2] = fmaf(t4[2], scp[mt][1][hb], acc[q][mt][2]);
-                    acc[q][mt][3] = fmaf(t4[3], scp[mt][1][hb], acc[q][mt][3]);
+                    ffma2_scalar(acc[q][mt][0], acc[q][mt][1], t4[0], t4[1], scb[mt][0]);
+                    ffma2_scalar(acc[q][mt][2], acc[q][mt][3], t4[2], t4[3], scb[mt][1]);
                   } else if constexpr (F == kINT4) {
                     mma_f16(tmp[q][mt], A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
                     mma_f16(tmp[q][mt], A[mt][1][0], A[mt][1][1], A[mt][1][2], A[mt][1][3], xv.z, xv.w);
