@@ -212,51 +212,29 @@ __device__ __forceinline__ float e8m0_to_f32(uint32_t v) {
   return __int_as_float(static_cast<int>(v << 23));
 }
 
-// E4M3 (FN) byte -> fp16 bits (exact: every finite E4M3 value is an fp16 value).
-__device__ __forceinline__ uint16_t e4m3_to_f16_bits(uint32_t b) {
-  const uint32_t s = (b >> 7) & 1u, e = (b >> 3) & 15u, m = b & 7u;
-  if (e == 15u && m == 7u) return 0x7e00u;  // NaN
-  uint32_t h;
-  if (e == 0u) {
-    // subnormal m/8 * 2^-6 = m * 2^-9 ; in fp16 that is a normal number for m>0
-    if (m == 0u) {
-      h = 0u;
-    } else {
-      // normalise: value = m * 2^-9, m in 1..7
-      int lz = __clz(m) - 29;           // leading zeros within 3 bits
-      uint32_t mm = (m << (lz + 1)) & 7u; // drop the leading one
-      int ex = -9 + (2 - lz);            // exponent of the leading one
-      h = (static_cast<uint32_t>(ex + 15) << 10) | (mm << 7);
-    }
-  } else {
-    h = ((e - 7u + 15u) << 10) | (m << 7);
-  }
-  return static_cast<uint16_t>((s << 15) | h);
+// Two E4M3 (FN) bytes (low byte, high byte of a 16-bit value) -> f16x2 with
+// the low byte's value in the low half (exact: every E4M3 value is an fp16
+// value), by the hardware conversion.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair16) {
+  uint32_t r;
+  asm("{\n .reg .b16 t;\n cvt.u16.u32 t, %1;\n cvt.rn.f16x2.e4m3x2 %0, t;\n}\n" : "=r"(r) : "r"(pair16));
+  return r;
 }
 
-// 8 INT4 codes (two's complement, one 32-bit word) -> four f16x2 words holding
-// exactly the integers q in [-8, 7].  Pairing: o0 = (n0, n4), o1 = (n1, n5),
-// o2 = (n2, n6), o3 = (n3, n7), where nI is nibble I counting from bit 0.
-// Uses f16 1024 + u (u = q + 8 in the mantissa) and subtracts 1032.
-__device__ __forceinline__ void int4x8_to_f16x8(uint32_t w, uint32_t& o0, uint32_t& o1, uint32_t& o2,
-                                                uint32_t& o3) {
-  const uint32_t u = w ^ 0x88888888u;  // q + 8 per nibble
-  const uint32_t magic = 0x64006400u;  // f16 (1024, 1024)
-  const uint32_t lo0 = (u & 0x000f000fu) | magic;         // 1024 + u0, 1024 + u4
-  const uint32_t hi0 = (u & 0x00f000f0u) | magic;         // 1024 + 16 u1, ...
-  const uint32_t lo1 = ((u >> 8) & 0x000f000fu) | magic;  // u2, u6
-  const uint32_t hi1 = ((u >> 8) & 0x00f000f0u) | magic;  // 16 u3, 16 u7
-  const __half2 k1032 = __half2half2(__ushort_as_half(0x6408u));  // 1032
-  const __half2 k72 = __half2half2(__ushort_as_half(0x5480u));    // 72
-  const __half2 k16th = __half2half2(__ushort_as_half(0x2c00u));  // 1/16
-  __half2 r0 = __hsub2(*reinterpret_cast<const __half2*>(&lo0), k1032);
-  __half2 r1 = __hfma2(*reinterpret_cast<const __half2*>(&hi0), k16th, __hneg2(k72));
-  __half2 r2 = __hsub2(*reinterpret_cast<const __half2*>(&lo1), k1032);
-  __half2 r3 = __hfma2(*reinterpret_cast<const __half2*>(&hi1), k16th, __hneg2(k72));
-  o0 = *reinterpret_cast<uint32_t*>(&r0);
-  o1 = *reinterpret_cast<uint32_t*>(&r1);
-  o2 = *reinterpret_cast<uint32_t*>(&r2);
-  o3 = *reinterpret_cast<uint32_t*>(&r3);
+// 8 INT4 codes (two's complement q in [-8, 7], one 32-bit word) -> four f16x2
+// words holding offset integers, one AND-XOR each: the even nibbles become
+// 1024 + (q + 8) and the odd nibbles 1024 + 16 (q + 8) (exact in fp16, whose
+// spacing at 1024 is 1).  Pairing: o0 = (n0, n4), o1 = (n1, n5), o2 = (n2, n6),
+// o3 = (n3, n7), nI being nibble I counting from bit 0.  The caller divides
+// the activations that meet odd nibbles by 16 and removes the constant part,
+// 1032 x (even) and 1152 x' (odd, x' = x / 16), per scale group.
+__device__ __forceinline__ void int4x8_to_f16x8_offset(uint32_t w, uint32_t& o0, uint32_t& o1, uint32_t& o2,
+                                                       uint32_t& o3) {
+  const uint32_t w8 = w >> 8;
+  o0 = (w & 0x000f000fu) ^ 0x64086408u;
+  o1 = (w & 0x00f000f0u) ^ 0x64806480u;
+  o2 = (w8 & 0x000f000fu) ^ 0x64086408u;
+  o3 = (w8 & 0x00f000f0u) ^ 0x64806480u;
 }
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __int_as_float(static_cast<int>(b << 16)); }

@@ -14,14 +14,15 @@
 //   stage 1: h = silu(x W_gate^T) * (x W_up^T)   (gate and up tiles paired)
 //   stage 2: y = h W_down^T
 //
-// Block = 8 consumer warps + 1 producer warp, one block per SM, persistent
+// Block = 8 consumer warps + 1 producer warp, two blocks per SM, persistent
 // over the work items.  The producer's elected lane issues TMA tiled loads
 // (128-row x 128-byte boxes, 128-byte swizzle) of the weights and of the
 // expert's activation rows into a ring of shared-memory stages, completing on
 // mbarriers.  Consumers decode the 4-bit codes to fp16 (E2M1 with the
-// hardware cvt, INT4 by the 1024-offset trick) and run m16n8k16 MMAs with
-// fp32 accumulation.  Block scales: MXFP4 (E8M0 per 32) and INT4 (bf16 per
-// 128) multiply the fp32 partial sums of their block; NVFP4 (E4M3 per 16)
+// hardware cvt; INT4 as offset integers 1024 + 16^j (q + 8), one AND-XOR per
+// pair, whose constant part is removed per scale group) and run m16n8k16 MMAs
+// with fp32 accumulation.  Block scales: MXFP4 (E8M0 per 32) and INT4 (bf16
+// per 128) multiply the fp32 partial sums of their block; NVFP4 (E4M3 per 16)
 // multiplies the fp16 weights (exact in fp16) and its fp32 global scale is
 // applied in the epilogue.  Within each 32-wide K block lane c of a quad
 // holds K = 8c..8c+7, i.e. the MMA's K order is a fixed permutation of the
@@ -29,9 +30,13 @@
 // weight rows) are read through the row order sigma(g) = (g>>1) | (g&1)<<2
 // inside each group of 8 so that the swizzled 16-byte reads are free of bank
 // conflicts; the epilogue maps columns (rows) back through the same sigma.
+// A full K chunk runs as straight-line code (every block and column group
+// known at compile time); only a ragged last chunk takes the guarded path.
 #include <cstdlib>
+#include <type_traits>
 
 #include "ffn_stream.cuh"
+#include "tc_ptx.cuh"
 #include "launch.cuh"
 #include "profile.cuh"
 
@@ -51,18 +56,19 @@ struct FmtTraits<kBF16> {
   static constexpr int kc = 64;     // K values per stage (128 bytes of a weight row)
   static constexpr int blk = 0;     // scale block (0: none)
   static constexpr int sbytes = 0;  // bytes per scale
+  static constexpr int kcpc = 1;    // 32-bit TMEM columns of scales per stage (unused without scales)
 };
 template <>
 struct FmtTraits<kMXFP4> {
-  static constexpr int kc = 256, blk = 32, sbytes = 1;
+  static constexpr int kc = 256, blk = 32, sbytes = 1, kcpc = 2;
 };
 template <>
 struct FmtTraits<kNVFP4> {
-  static constexpr int kc = 256, blk = 16, sbytes = 1;
+  static constexpr int kc = 256, blk = 16, sbytes = 1, kcpc = 4;
 };
 template <>
 struct FmtTraits<kINT4> {
-  static constexpr int kc = 256, blk = 128, sbytes = 2;
+  static constexpr int kc = 256, blk = 128, sbytes = 2, kcpc = 1;
 };
 
 __device__ __forceinline__ int sigma8(int g) { return (g >> 1) | ((g & 1) << 2); }
@@ -143,6 +149,7 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
   constexpr int W_BYTES = kRowsPerStage * kLine;
   constexpr int X_BYTES = NXBOX * XCOLS * kLine;
   constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
+  constexpr int kCpc = Tr::kcpc;                // TMEM scale columns per K chunk
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
 
@@ -151,26 +158,19 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + kMaxStages;
-  uint64_t* sfull = empty + kMaxStages;
-  uint64_t* sempty = sfull + 2;
-  volatile int* s_abort = reinterpret_cast<volatile int*>(sempty + 2);
-  int* s_ngroups = reinterpret_cast<int*>(sempty + 2) + 1;
-  int* s_offs = reinterpret_cast<int*>(sempty + 2) + 4;  // [E+1]
-  int* s_gitem = s_offs + (a.E + 4);                     // [groups+1]
-  int* s_gexp = s_gitem + (a.E + a.n_shared + 4);        // [groups]
-  const int hdr = stream_hdr_bytes(a.E, a.n_shared);
-  uint8_t* s_scale = smem + hdr;
-  uint8_t* s_stage = s_scale + a.n_scale_buf * a.smem_scale_bytes;
+  volatile int* s_abort = reinterpret_cast<volatile int*>(empty + kMaxStages);
+  int* s_ngroups = reinterpret_cast<int*>(empty + kMaxStages) + 1;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(empty + kMaxStages) + 2;
+  int* s_offs = reinterpret_cast<int*>(empty + kMaxStages) + 4;  // [E+1]
+  int* s_gitem = s_offs + (a.E + 4);                             // [groups+1]
+  int* s_gexp = s_gitem + (a.E + a.n_shared + 4);                // [groups]
+  uint8_t* s_stage = smem + stream_hdr_bytes(a.E, a.n_shared);
 
   const int E = a.E;
   if (tid == 0) {
     for (int i = 0; i < a.n_stages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], kConsumerWarps);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sfull[i], 1);
-      mbar_init(&sempty[i], kConsumerWarps);
     }
     *s_abort = 0;
     fence_barrier_init();
@@ -181,6 +181,13 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
   const int rows_per_item = kGateUp ? kRowsPerStage / 2 : kRowsPerStage;
   const int ntile = ceil_div(a.N, rows_per_item);
   if (warp == 0) {
+    // Block scales live in tensor memory while an item runs: lane i of warp w
+    // keeps the scales of one weight row in TMEM lane 32 (w % 4) + i, columns
+    // [(w / 4) C, (w / 4 + 1) C).  Two blocks per SM use at most 2 x 256 columns.
+    if (Tr::blk) {
+      tc::tmem_alloc(s_tmem, (uint32_t)a.tmem_alloc);
+      tc::tmem_relinquish();
+    }
     int ng = 0, items = 0;
     for (int sh = 0; sh < a.n_shared; ++sh) {
       if (lane == 0) {
@@ -223,14 +230,17 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
       *s_ngroups = ng;
     }
   }
+  tc::fence_before_sync();
   __syncthreads();
+  tc::fence_after_sync();
   const int ngroups = *s_ngroups;
   const int n_items = s_gitem[ngroups];
   const int K = a.K;
   const int srow = Tr::blk ? (K / Tr::blk) * Tr::sbytes : 0;
   const int nchunks = ceil_div(K, KC);
   const int nstage = a.n_stages;
-  const int nsb = a.n_scale_buf;
+  const int n_sslots = Tr::blk ? a.n_sslots : 0;  // ring stages carrying an item's block scales
+  const int slot_warps = kConsumerWarps / (n_sslots ? n_sslots : 1);
   const int x_row_bytes = K * 2;
 
   if (warp == kConsumerWarps) {
@@ -239,64 +249,67 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
       prefetch_tmap(&a.tm_w);
       prefetch_tmap(&a.tm_x);
       if (a.n_shared) prefetch_tmap(&a.tm_wsh);
-      const uint64_t pol_w = a.w_l2_normal ? l2_evict_normal_policy() : l2_evict_first_policy();
+      const uint64_t pol_w = a.w_l2_first ? l2_evict_first_policy() : l2_evict_normal_policy();
       const uint64_t pol_x = l2_evict_last_policy();
       uint32_t cnt = 0;
-      int item_no = 0;
-      for (int item = blockIdx.x; item < n_items && !*s_abort; item += gridDim.x, ++item_no) {
+      for (int item = blockIdx.x; item < n_items && !*s_abort; item += gridDim.x) {
         const Item it = decode_item<F>(a, item, ntile, s_gitem, s_gexp, ngroups, s_offs);
         const int r0 = it.tile * rows_per_item;
         const int nrows = min(rows_per_item, a.N - r0);
-        const int sb = item_no % nsb;
-        const uint32_t suse = item_no / nsb;
-        const int sc_at = (nsb == 2) ? 0 : min(nstage - 1, nchunks - 1);
         const CUtensorMap* tw = it.shared_idx >= 0 ? &a.tm_wsh : &a.tm_w;
+        // The item's block scales first, in n_sslots ring stages: stage j holds
+        // the rows of consumer warps [j * slot_warps, (j + 1) * slot_warps) --
+        // gate rows then up rows (stage 1), or 32 rows per warp (stage 2) --
+        // each a contiguous range of the row-major scale matrix.
+        for (int j = 0; j < n_sslots && !*s_abort; ++j) {
+          const int s = cnt % nstage;
+          if (!mbar_wait(&empty[s], ((cnt / nstage) & 1u) ^ 1u)) {
+            *s_abort = 1;
+            break;
+          }
+          uint8_t* dst = s_stage + s * STAGE_BYTES;
+          const int wrows = kGateUp ? 16 : 32;  // scale rows per warp and matrix half
+          const int first = j * slot_warps * wrows;
+          const int cnt_rows = max(0, min(nrows - first, slot_warps * wrows));
+          const uint32_t bytes = (uint32_t)(cnt_rows * srow);
+          mbar_arrive_expect_tx(&full[s], it.valid ? bytes * (kGateUp ? 2u : 1u) : 0u);
+          if (it.valid && cnt_rows > 0) {
+            bulk_g2s(dst, it.sbase + (int64_t)(r0 + first) * srow, bytes, &full[s]);
+            if (kGateUp)
+              bulk_g2s(dst + slot_warps * wrows * srow, it.sbase + (int64_t)(a.N + r0 + first) * srow, bytes,
+                       &full[s]);
+          }
+          ++cnt;
+        }
         // boxes of weight rows: stage 1 gate rows r0.. and up rows N+r0..; stage 2 rows r0.., r0+128..
         const int nbox_w = kGateUp ? 2 : (nrows > kBoxRows ? 2 : 1);
-        for (int pass = it.pass; pass == it.pass && !*s_abort; ++pass) {
-          const int c0 = pass * XCOLS;
-          for (int ch = 0; ch < nchunks; ++ch) {
-            if (Tr::blk && ch == sc_at) {
-              if (!mbar_wait(&sempty[sb], (suse & 1u) ^ 1u)) {
-                *s_abort = 1;
-                break;
-              }
-              const uint32_t bytes = (uint32_t)(nrows * srow);
-              mbar_arrive_expect_tx(&sfull[sb], it.valid ? bytes * (kGateUp ? 2u : 1u) : 0u);
-              if (it.valid) {
-                uint8_t* dst = s_scale + sb * a.smem_scale_bytes;
-                bulk_g2s(dst, it.sbase + (int64_t)r0 * srow, bytes, &sfull[sb]);
-                if (kGateUp)
-                  bulk_g2s(dst + rows_per_item * srow, it.sbase + (int64_t)(a.N + r0) * srow, bytes, &sfull[sb]);
-              }
-            }
-            const int s = cnt % nstage;
-            if (!mbar_wait(&empty[s], ((cnt / nstage) & 1u) ^ 1u)) {
-              *s_abort = 1;
-              break;
-            }
-            uint8_t* st_w = s_stage + s * STAGE_BYTES;
-            uint8_t* st_x = st_w + W_BYTES;
-            const int kb = ch * kLine;                 // byte offset inside a weight row
-            const int xb0 = ch * KC * 2;               // byte offset inside an activation row
-            int nxb = 0;
-            for (int q = 0; q < NXBOX; ++q) nxb += (xb0 + q * kLine < x_row_bytes) ? 1 : 0;
-            const uint32_t bytes =
-                it.valid ? (uint32_t)(nbox_w * kBoxRows * kLine + nxb * XCOLS * kLine) : 0u;
-            mbar_arrive_expect_tx(&full[s], bytes);
-            if (it.valid) {
-              if (kGateUp) {
-                tma_load_3d(st_w, tw, kb, r0, it.phys, &full[s], pol_w);
-                tma_load_3d(st_w + kBoxRows * kLine, tw, kb, a.N + r0, it.phys, &full[s], pol_w);
-              } else {
-                tma_load_3d(st_w, tw, kb, r0, it.phys, &full[s], pol_w);
-                if (nbox_w == 2) tma_load_3d(st_w + kBoxRows * kLine, tw, kb, r0 + kBoxRows, it.phys, &full[s], pol_w);
-              }
-              for (int q = 0; q < nxb; ++q)
-                tma_load_2d(st_x + q * XCOLS * kLine, &a.tm_x, xb0 + q * kLine, it.xrow0 + c0, &full[s], pol_x);
-            }
-            ++cnt;
+        const int c0 = it.pass * XCOLS;
+        for (int ch = 0; ch < nchunks && !*s_abort; ++ch) {
+          const int s = cnt % nstage;
+          if (!mbar_wait(&empty[s], ((cnt / nstage) & 1u) ^ 1u)) {
+            *s_abort = 1;
+            break;
           }
+          uint8_t* st_w = s_stage + s * STAGE_BYTES;
+          uint8_t* st_x = st_w + W_BYTES;
+          const int kb = ch * kLine;                 // byte offset inside a weight row
+          const int xb0 = ch * KC * 2;               // byte offset inside an activation row
+          int nxb = 0;
+          for (int q = 0; q < NXBOX; ++q) nxb += (xb0 + q * kLine < x_row_bytes) ? 1 : 0;
+          const uint32_t bytes = it.valid ? (uint32_t)(nbox_w * kBoxRows * kLine + nxb * XCOLS * kLine) : 0u;
+          mbar_arrive_expect_tx(&full[s], bytes);
+          if (it.valid) {
+            if (kGateUp) {
+              tma_load_3d(st_w, tw, kb, r0, it.phys, &full[s], pol_w);
+              tma_load_3d(st_w + kBoxRows * kLine, tw, kb, a.N + r0, it.phys, &full[s], pol_w);
+            } else {
+              tma_load_3d(st_w, tw, kb, r0, it.phys, &full[s], pol_w);
+              if (nbox_w == 2) tma_load_3d(st_w + kBoxRows * kLine, tw, kb, r0 + kBoxRows, it.phys, &full[s], pol_w);
+            }
+            for (int q = 0; q < nxb; ++q)
+              tma_load_2d(st_x + q * XCOLS * kLine, &a.tm_x, xb0 + q * kLine, it.xrow0 + c0, &full[s], pol_x);
+          }
+          ++cnt;
         }
       }
       // Let every load this lane issued land before the block can exit.
@@ -309,222 +322,309 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
   // ======================================================= consumer warps
   const int g = lane >> 2, c = lane & 3;
   const int sg = sigma8(g);
+  // Rows of this warp's two m16 tiles inside a stage (multiples of 16).
+  const int m0 = kGateUp ? warp * 16 : warp * 32;
+  constexpr int kDm = kGateUp ? kRowsPerStage / 2 : 16;  // second m-tile, rows below the first
+  // Stage-relative byte offsets of this lane's operands.  A 128-byte row r
+  // keeps its 16-byte granule j at ((j ^ (r & 7)) << 4) (TMA 128-byte
+  // swizzle).  For every row this lane reads, r & 7 is g (4-bit codes) or
+  // sigma(g) (bf16 weights, activations), so the granule of block b is one XOR
+  // away from the lane's block-0 address, and rows g + 8 and the second
+  // m-tile sit at fixed distances from it.
+  const uint32_t w_lane = (F == kBF16) ? (uint32_t)(m0 + sg) * kLine + ((uint32_t)(c ^ sg) << 4)
+                                       : (uint32_t)(m0 + g) * kLine + ((uint32_t)g << 4) + 4u * c;
+  constexpr uint32_t kRow8 = 8 * kLine;
+  constexpr uint32_t kDmBytes = kDm * kLine;
+  const uint32_t x_lane = W_BYTES + (uint32_t)sg * kLine + ((uint32_t)(c ^ sg) << 4);
+  // Block scales: lane c of a quad owns the scale row of m-tile c>>1, row
+  // g + 8(c&1) (each lane of the warp a different row), keeps it in TMEM, and
+  // hands the quad's other lanes what they need through shuffles.
+  const uint32_t t_row = Tr::blk ? *s_tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)((warp >> 2) * a.tmem_cols)
+                                 : 0u;
+  // the owned row inside its scale stage (gate rows of the stage's warps, then up rows)
+  const int s_wl = warp % slot_warps;
+  const int s_row = kGateUp ? ((c >> 1) ? 16 * slot_warps : 0) + 16 * s_wl + g + 8 * (c & 1)
+                            : 32 * s_wl + 16 * (c >> 1) + g + 8 * (c & 1);
   uint32_t cnt = 0;
-  int item_no = 0;
   const uint32_t stage0 = smem_u32(s_stage);
-  const uint32_t scale0 = smem_u32(s_scale);
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++item_no) {
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     const Item it = decode_item<F>(a, item, ntile, s_gitem, s_gexp, ngroups, s_offs);
     const int r0 = it.tile * rows_per_item;
     const int nrows = min(rows_per_item, a.N - r0);
-    const int sb = item_no % nsb;
-    const uint32_t suse = item_no / nsb;
-    // smem rows of this warp's two m16 tiles
-    const int m0 = kGateUp ? warp * 16 : warp * 32;
-    const int m1 = kGateUp ? rows_per_item + warp * 16 : warp * 32 + 16;
     const bool active = it.valid && (kGateUp ? (warp * 16 < nrows) : (warp * 32 < nrows));
-    if (Tr::blk) {
-      if (!mbar_wait(&sfull[sb], suse & 1u)) *s_abort = 1;
-    }
-    const uint32_t sc_base = scale0 + sb * a.smem_scale_bytes;
-    for (int pass = it.pass; pass == it.pass; ++pass) {
-      const int c0 = pass * XCOLS;
-      const int ncols = min(XCOLS, it.n_cols - c0);
-      const int ng_act = ceil_div(ncols, 8);
-      float acc[NG][2][4];
+    const int c0 = it.pass * XCOLS;
+    const int ncols = min(XCOLS, it.n_cols - c0);
+    const int ng_act = ceil_div(ncols, 8);
+    // --------------------------------------------- block scales -> TMEM
+    for (int j = 0; j < n_sslots; ++j) {
+      const int s = cnt % nstage;
+      if (*s_abort || !mbar_wait(&full[s], (cnt / nstage) & 1u)) {
+        *s_abort = 1;
+        break;
+      }
+      if (active && ncols > 0 && warp / slot_warps == j) {
+        const uint32_t ra = stage0 + s * STAGE_BYTES + s_row * srow;
+        for (int cb = 0; cb < a.tmem_cols; cb += 4) {
+          uint32_t v[4];
 #pragma unroll
-      for (int q = 0; q < NG; ++q)
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-          for (int r = 0; r < 4; ++r) acc[q][mt][r] = 0.f;
-      float tmp[NG][2][4];  // INT4 group partials
-      for (int ch = 0; ch < nchunks; ++ch) {
-        const int s = cnt % nstage;
-        if (*s_abort || !mbar_wait(&full[s], (cnt / nstage) & 1u)) {
-          *s_abort = 1;
-          break;
-        }
-        if (active && ncols > 0) {
-          const uint32_t wst = stage0 + s * STAGE_BYTES;
-          const uint32_t xst = wst + W_BYTES;
-          const int nblk = min(KC, K - ch * KC) / 32;
-          // MXFP4 block scales of this chunk: the four lanes of a quad need the
-          // same four rows, so lane c converts the chunk's eight scales of one
-          // of them (m-tile c>>1, row g + 8(c&1)), two per 16-bit load, and the
-          // quad shares them through shuffles.
-          float sc8[KC / 32];
-          if constexpr (F == kMXFP4) {
-            const bool pair_aligned = (srow & 1) == 0;
-            const uint32_t ad0 = sc_base + (((c >> 1) ? m1 : m0) + g + 8 * (c & 1)) * srow + (ch * KC) / 32;
-#pragma unroll
-            for (int p = 0; p < KC / 64; ++p) {
-              uint32_t v = 0x7f7fu;  // past the row's last block: unused
-              if (2 * p < nblk) v = pair_aligned ? lds16(ad0 + 2 * p) : (lds8(ad0 + 2 * p) | (lds8(ad0 + 2 * p + 1) << 8));
-              e8m0x2_to_f32x2(v, sc8[2 * p], sc8[2 * p + 1]);
+          for (int t = 0; t < 4; ++t) {
+            const int b0 = 4 * (cb + t);
+            if (b0 + 4 <= srow) {
+              if ((srow & 3) == 0) v[t] = lds32(ra + b0);
+              else if ((srow & 1) == 0) v[t] = lds16(ra + b0) | (lds16(ra + b0 + 2) << 16);
+              else v[t] = lds8(ra + b0) | (lds8(ra + b0 + 1) << 8) | (lds8(ra + b0 + 2) << 16) | (lds8(ra + b0 + 3) << 24);
+            } else {
+              v[t] = 0;
+              for (int u = 0; u < 4 && b0 + u < srow; ++u) v[t] |= lds8(ra + b0 + u) << (8 * u);
             }
           }
+          tc::tmem_st_32x32b_x4(t_row + cb, v);
+        }
+        tc::tmem_st_wait();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      ++cnt;
+    }
+    if (*s_abort) break;
+    float acc[NG][2][4];
 #pragma unroll
-          for (int bp = 0; bp < KC / 32; bp += 2) {
-            if (bp >= nblk) break;
+    for (int q = 0; q < NG; ++q)
 #pragma unroll
-            for (int hb = 0; hb < 2; ++hb) {
-            const int b = bp + hb;
-            if (b >= nblk) break;
-            float scb[2][2];  // MXFP4 scale of block b for [m-tile][row g / g+8]
-            if constexpr (F == kMXFP4) {
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) acc[q][mt][r] = 0.f;
+    float tmp[NG][2][4];  // INT4 group partials
+    float gbias[NG][2];   // INT4 constant part of the group's partials, per column
+    const int n_grp = K / 128;
+    for (int ch = 0; ch < nchunks; ++ch) {
+      const int s = cnt % nstage;
+      const bool work = active && ncols > 0;
+      // this chunk's scales of the owned row (issued before the wait for the stage)
+      uint32_t sv[4] = {0u, 0u, 0u, 0u};
+      if constexpr (Tr::blk != 0) {
+        if (work) tc::tmem_ld_cols<kCpc>(t_row + ch * kCpc, sv);
+      }
+      if (*s_abort || !mbar_wait(&full[s], (cnt / nstage) & 1u)) {
+        if constexpr (Tr::blk != 0) {
+          if (work) tc::tmem_ld_wait<kCpc>(sv);
+        }
+        *s_abort = 1;
+        break;
+      }
+      if (work) {
+        if constexpr (Tr::blk != 0) tc::tmem_ld_wait<kCpc>(sv);
+        const uint32_t wst = stage0 + s * STAGE_BYTES;
+        const uint32_t wa0 = wst + w_lane;
+        const uint32_t xa0 = wst + x_lane;  // activation granule of even blocks
+        const uint32_t xa1 = xa0 ^ 64u;     // odd blocks: granule 4 + c
+        const int nblk = min(KC, K - ch * KC) / 32;
+        // MXFP4: the owned row's eight scales of this chunk, as fp32
+        float sc8[KC / 32];
+        if constexpr (F == kMXFP4) {
+#pragma unroll
+          for (int p = 0; p < KC / 64; ++p) e8m0x2_to_f32x2((sv[p >> 1] >> (16 * (p & 1))) & 0xffffu, sc8[2 * p], sc8[2 * p + 1]);
+        }
+        // One 32-wide K block b for NQ column groups; with kGuard the groups
+        // at or beyond ng_act are skipped at run time.
+        auto block = [&](const int b, auto nq_tag, auto guard_tag) {
+          constexpr int NQ = decltype(nq_tag)::value;
+          constexpr bool kGuard = decltype(guard_tag)::value;
+          [[maybe_unused]] float scb[2][2];  // MXFP4 scale of block b for [m-tile][row g / g+8]
+          if constexpr (F == kMXFP4) {
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+              for (int hr = 0; hr < 2; ++hr)
+                scb[mt][hr] = __shfl_sync(0xffffffffu, sc8[b], (lane & ~3) | (2 * mt + hr));
+          }
+          uint32_t A[2][2][4];  // [m-tile][k16 tile][reg]
+          if constexpr (F == kBF16) {
+            const uint32_t wa = wa0 ^ ((uint32_t)b << 6);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+              const uint4 lo = lds128(wa + mt * kDmBytes);
+              const uint4 hi = lds128(wa + mt * kDmBytes + kRow8);
+              A[mt][0][0] = lo.x; A[mt][0][1] = hi.x; A[mt][0][2] = lo.y; A[mt][0][3] = hi.y;
+              A[mt][1][0] = lo.z; A[mt][1][1] = hi.z; A[mt][1][2] = lo.w; A[mt][1][3] = hi.w;
+            }
+          } else {
+            const uint32_t wa = wa0 ^ ((uint32_t)b << 4);
+            // NVFP4: the two 16-block scales of block b of each owned row sit in
+            // one 16-bit half of the row's chunk word b>>1; this lane's 8 values
+            // lie in 16-block 2b + (c>>1)
+            [[maybe_unused]] uint32_t nv[2][2];
+            if constexpr (F == kNVFP4) {
 #pragma unroll
               for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
                 for (int hr = 0; hr < 2; ++hr)
-                  scb[mt][hr] = __shfl_sync(0xffffffffu, sc8[b], (lane & ~3) | (2 * mt + hr));
+                  nv[mt][hr] = __shfl_sync(0xffffffffu, sv[b >> 1], (lane & ~3) | (2 * mt + hr)) >>
+                               (16 * (b & 1) + 8 * (c >> 1));
             }
-            uint32_t A[2][2][4];  // [m-tile][k16 tile][reg]
-            if constexpr (F == kBF16) {
 #pragma unroll
-              for (int mt = 0; mt < 2; ++mt) {
-                const int mr = mt ? m1 : m0;
-                const uint32_t gran = (uint32_t)((4 * b + c) ^ sg) << 4;
-                const uint4 lo = lds128(wst + (mr + sg) * kLine + gran);
-                const uint4 hi = lds128(wst + (mr + 8 + sg) * kLine + gran);
-                A[mt][0][0] = lo.x; A[mt][0][1] = hi.x; A[mt][0][2] = lo.y; A[mt][0][3] = hi.y;
-                A[mt][1][0] = lo.z; A[mt][1][1] = hi.z; A[mt][1][2] = lo.w; A[mt][1][3] = hi.w;
+            for (int mt = 0; mt < 2; ++mt) {
+              const uint32_t wlo = lds32(wa + mt * kDmBytes);
+              const uint32_t whi = lds32(wa + mt * kDmBytes + kRow8);
+              uint32_t l0, l1, l2, l3, h0, h1, h2, h3;
+              if constexpr (F == kINT4) {
+                int4x8_to_f16x8_offset(wlo, l0, l1, l2, l3);
+                int4x8_to_f16x8_offset(whi, h0, h1, h2, h3);
+              } else {
+                e2m1x8_to_f16x8(wlo, l0, l1, l2, l3);
+                e2m1x8_to_f16x8(whi, h0, h1, h2, h3);
               }
-            } else {
-#pragma unroll
-              for (int mt = 0; mt < 2; ++mt) {
-                const int mr = mt ? m1 : m0;
-                const uint32_t off = ((uint32_t)(b ^ g) << 4) + 4 * c;
-                const uint32_t wlo = lds32(wst + (mr + g) * kLine + off);
-                const uint32_t whi = lds32(wst + (mr + g + 8) * kLine + off);
-                uint32_t l0, l1, l2, l3, h0, h1, h2, h3;
-                if constexpr (F == kINT4) {
-                  int4x8_to_f16x8(wlo, l0, l1, l2, l3);
-                  int4x8_to_f16x8(whi, h0, h1, h2, h3);
-                } else {
-                  e2m1x8_to_f16x8(wlo, l0, l1, l2, l3);
-                  e2m1x8_to_f16x8(whi, h0, h1, h2, h3);
-                }
-                if constexpr (F == kNVFP4) {
-                  // this lane's 8 values share one 16-block per row
-                  const int nb = (ch * KC + b * 32 + 8 * c) >> 4;
-                  const uint32_t slo = e4m3_to_f16_bits(lds8(sc_base + (mr + g) * srow + nb));
-                  const uint32_t shi = e4m3_to_f16_bits(lds8(sc_base + (mr + g + 8) * srow + nb));
-                  const uint32_t slo2 = slo | (slo << 16), shi2 = shi | (shi << 16);
-                  l0 = hmul2_u32(l0, slo2); l1 = hmul2_u32(l1, slo2); l2 = hmul2_u32(l2, slo2); l3 = hmul2_u32(l3, slo2);
-                  h0 = hmul2_u32(h0, shi2); h1 = hmul2_u32(h1, shi2); h2 = hmul2_u32(h2, shi2); h3 = hmul2_u32(h3, shi2);
-                }
-                A[mt][0][0] = l0; A[mt][0][1] = h0; A[mt][0][2] = l1; A[mt][0][3] = h1;
-                A[mt][1][0] = l2; A[mt][1][1] = h2; A[mt][1][2] = l3; A[mt][1][3] = h3;
+              if constexpr (F == kNVFP4) {
+                const uint32_t pair = (nv[mt][0] & 0xffu) | ((nv[mt][1] & 0xffu) << 8);
+                const uint32_t s2 = e4m3x2_to_f16x2(pair);
+                const uint32_t slo2 = __byte_perm(s2, 0u, 0x1010), shi2 = __byte_perm(s2, 0u, 0x3232);
+                l0 = hmul2_u32(l0, slo2); l1 = hmul2_u32(l1, slo2); l2 = hmul2_u32(l2, slo2); l3 = hmul2_u32(l3, slo2);
+                h0 = hmul2_u32(h0, shi2); h1 = hmul2_u32(h1, shi2); h2 = hmul2_u32(h2, shi2); h3 = hmul2_u32(h3, shi2);
               }
-            }
-            if constexpr (F == kINT4) {
-              if ((b & 3) == 0) {
-#pragma unroll
-                for (int q = 0; q < NG; ++q)
-#pragma unroll
-                  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) tmp[q][mt][r] = 0.f;
-              }
-            }
-            // activation fragment address: box b/2, granule (b&1)*4+c of row q*8+sigma(g)
-            const uint32_t xoff = (uint32_t)(b >> 1) * (XCOLS * kLine) + (uint32_t)sg * kLine +
-                                  ((uint32_t)(((hb << 2) + c) ^ sg) << 4);
-#pragma unroll
-            for (int q = 0; q < NG; ++q) {
-              if (q < ng_act) {
-                const uint4 xv = lds128(xst + xoff + q * 8 * kLine);
-#pragma unroll
-                for (int mt = 0; mt < 2; ++mt) {
-                  if constexpr (F == kMXFP4) {
-                    float t4[4];
-                    mma_f16_z(t4, A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
-                    mma_f16(t4, A[mt][1][0], A[mt][1][1], A[mt][1][2], A[mt][1][3], xv.z, xv.w);
-                    ffma2_scalar(acc[q][mt][0], acc[q][mt][1], t4[0], t4[1], scb[mt][0]);
-                    ffma2_scalar(acc[q][mt][2], acc[q][mt][3], t4[2], t4[3], scb[mt][1]);
-                  } else if constexpr (F == kINT4) {
-                    mma_f16(tmp[q][mt], A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
-                    mma_f16(tmp[q][mt], A[mt][1][0], A[mt][1][1], A[mt][1][2], A[mt][1][3], xv.z, xv.w);
-                  } else if constexpr (F == kNVFP4) {
-                    mma_f16(acc[q][mt], A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
-                    mma_f16(acc[q][mt], A[mt][1][0], A[mt][1][1], A[mt][1][2], A[mt][1][3], xv.z, xv.w);
-                  } else {
-                    mma_bf16(acc[q][mt], A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
-                    mma_bf16(acc[q][mt], A[mt][1][0], A[mt][1][1], A[mt][1][2], A[mt][1][3], xv.z, xv.w);
-                  }
-                }
-              }
-            }
-            if constexpr (F == kINT4) {
-              if ((b & 3) == 3 || b == nblk - 1) {
-                const int grp = (ch * KC + b * 32) / 128;
-#pragma unroll
-                for (int mt = 0; mt < 2; ++mt) {
-                  const int mr = mt ? m1 : m0;
-                  const float s_lo = bf16_bits_to_f32(lds16(sc_base + (mr + g) * srow + 2 * grp));
-                  const float s_hi = bf16_bits_to_f32(lds16(sc_base + (mr + g + 8) * srow + 2 * grp));
-#pragma unroll
-                  for (int q = 0; q < NG; ++q) {
-                    acc[q][mt][0] = fmaf(tmp[q][mt][0], s_lo, acc[q][mt][0]);
-                    acc[q][mt][1] = fmaf(tmp[q][mt][1], s_lo, acc[q][mt][1]);
-                    acc[q][mt][2] = fmaf(tmp[q][mt][2], s_hi, acc[q][mt][2]);
-                    acc[q][mt][3] = fmaf(tmp[q][mt][3], s_hi, acc[q][mt][3]);
-                  }
-                }
-              }
-            }
+              A[mt][0][0] = l0; A[mt][0][1] = h0; A[mt][0][2] = l1; A[mt][0][3] = h1;
+              A[mt][1][0] = l2; A[mt][1][1] = h2; A[mt][1][2] = l3; A[mt][1][3] = h3;
             }
           }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-        ++cnt;
-      }
-      if (*s_abort) break;
-      // ---------------------------------------------------------- epilogue
-      if (active && ncols > 0) {
+          if constexpr (F == kINT4) {
+            // constant part of this 128-wide group's offset products, per column
+            if ((b & 3) == 0) {
+              const int grp = (ch * KC + b * 32) / 128;
 #pragma unroll
-        for (int q = 0; q < NG; ++q) {
-          if (q < ng_act) {
+              for (int q = 0; q < NQ; ++q) {
+                if (kGuard && q >= ng_act) break;
 #pragma unroll
-            for (int hc = 0; hc < 2; ++hc) {
-              const int col = c0 + q * 8 + sigma8(2 * c + hc);  // activation row inside the expert
-              if (col < it.n_cols) {
-                const int xrow = it.xrow0 + col;
-                float f = it.gscale;
-                if (F != kBF16) f = ldexpf(f, __ldg(a.xexp + xrow));
-                // weight rows held by this lane: (row g, row g+8) of each m-tile (bf16: sigma(g))
-                const int wr = (F == kBF16) ? sg : g;
-                if (kGateUp) {
-                  __nv_bfloat16* o = a.out_routed + (int64_t)xrow * a.N + r0 + warp * 16;
-#pragma unroll
-                  for (int hr = 0; hr < 2; ++hr) {
-                    const float gt = acc[q][0][hr * 2 + hc] * f;
-                    const float up = acc[q][1][hr * 2 + hc] * f;
-                    const float h = gt / (1.f + expf(-gt)) * up;
-                    o[wr + 8 * hr] = __float2bfloat16_rn(h);
-                  }
-                } else {
-                  __nv_bfloat16* o = it.shared_idx >= 0
-                                         ? a.out_shared + ((int64_t)it.shared_idx * a.T + col) * a.N
-                                         : a.out_routed + (int64_t)xrow * a.N;
-#pragma unroll
-                  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                    for (int hr = 0; hr < 2; ++hr)
-                      o[r0 + warp * 32 + mt * 16 + wr + 8 * hr] = __float2bfloat16_rn(acc[q][mt][hr * 2 + hc] * f);
+                for (int hc = 0; hc < 2; ++hc) {
+                  const int col = c0 + q * 8 + sigma8(2 * c + hc);
+                  const int row = it.xrow0 + (col < it.n_cols ? col : 0);
+                  gbias[q][hc] = __ldg(a.xbias + (int64_t)row * n_grp + grp);
                 }
+              }
+            }
+          }
+          // activation fragment: box b/2, granule (b&1)*4 + c of row q*8 + sigma(g)
+          const uint32_t xa = ((b & 1) ? xa1 : xa0) + (uint32_t)(b >> 1) * (XCOLS * kLine);
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) {
+            if (kGuard && q >= ng_act) break;
+            const uint4 xv = lds128(xa + q * 8 * kLine);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+              if constexpr (F == kMXFP4) {
+                float t4[4];
+                mma_f16_z(t4, A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
+                mma_f16(t4, A[mt][1][0], A[mt][1][1], A[mt][1][2], A[mt][1][3], xv.z, xv.w);
+                ffma2_scalar(acc[q][mt][0], acc[q][mt][1], t4[0], t4[1], scb[mt][0]);
+                ffma2_scalar(acc[q][mt][2], acc[q][mt][3], t4[2], t4[3], scb[mt][1]);
+              } else if constexpr (F == kINT4) {
+                if ((b & 3) == 0)
+                  mma_f16_z(tmp[q][mt], A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
+                else
+                  mma_f16(tmp[q][mt], A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
+                mma_f16(tmp[q][mt], A[mt][1][0], A[mt][1][1], A[mt][1][2], A[mt][1][3], xv.z, xv.w);
+              } else if constexpr (F == kNVFP4) {
+                mma_f16(acc[q][mt], A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
+                mma_f16(acc[q][mt], A[mt][1][0], A[mt][1][1], A[mt][1][2], A[mt][1][3], xv.z, xv.w);
+              } else {
+                mma_bf16(acc[q][mt], A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
+                mma_bf16(acc[q][mt], A[mt][1][0], A[mt][1][1], A[mt][1][2], A[mt][1][3], xv.z, xv.w);
+              }
+            }
+          }
+          if constexpr (F == kINT4) {
+            // end of a 128-wide scale group (or of the row): scale and accumulate
+            if ((b & 3) == 3 || b == nblk - 1) {
+              const int gi = b >> 2;  // group inside the chunk: bf16 half gi of the chunk word
+#pragma unroll
+              for (int mt = 0; mt < 2; ++mt) {
+                const uint32_t wlo = __shfl_sync(0xffffffffu, sv[0], (lane & ~3) | (2 * mt));
+                const uint32_t whi = __shfl_sync(0xffffffffu, sv[0], (lane & ~3) | (2 * mt + 1));
+                const float s_lo = __uint_as_float(gi ? (wlo & 0xffff0000u) : (wlo << 16));
+                const float s_hi = __uint_as_float(gi ? (whi & 0xffff0000u) : (whi << 16));
+#pragma unroll
+                for (int q = 0; q < NQ; ++q) {
+                  if (kGuard && q >= ng_act) break;
+                  const float t0 = tmp[q][mt][0] - gbias[q][0], t1 = tmp[q][mt][1] - gbias[q][1];
+                  const float t2 = tmp[q][mt][2] - gbias[q][0], t3 = tmp[q][mt][3] - gbias[q][1];
+                  ffma2_scalar(acc[q][mt][0], acc[q][mt][1], t0, t1, s_lo);
+                  ffma2_scalar(acc[q][mt][2], acc[q][mt][3], t2, t3, s_hi);
+                }
+              }
+            }
+          }
+        };
+        using IFull = std::integral_constant<int, NG>;
+        using IOne = std::integral_constant<int, 1>;
+        if (nblk == KC / 32) {
+          // full chunk: straight-line code, every block and column group static
+          if (ng_act >= NG) {
+#pragma unroll
+            for (int b = 0; b < KC / 32; ++b) block(b, IFull{}, std::false_type{});
+          } else if (NG > 1 && ng_act == 1) {
+#pragma unroll
+            for (int b = 0; b < KC / 32; ++b) block(b, IOne{}, std::false_type{});
+          } else {
+#pragma unroll
+            for (int b = 0; b < KC / 32; ++b) block(b, IFull{}, std::true_type{});
+          }
+        } else {
+#pragma unroll
+          for (int b = 0; b < KC / 32; ++b) {
+            if (b >= nblk) break;
+            block(b, IFull{}, std::true_type{});
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      ++cnt;
+    }
+    if (*s_abort) break;
+    // ---------------------------------------------------------- epilogue
+    if (active && ncols > 0) {
+#pragma unroll
+      for (int q = 0; q < NG; ++q) {
+        if (q < ng_act) {
+#pragma unroll
+          for (int hc = 0; hc < 2; ++hc) {
+            const int col = c0 + q * 8 + sigma8(2 * c + hc);  // activation row inside the expert
+            if (col < it.n_cols) {
+              const int xrow = it.xrow0 + col;
+              float f = it.gscale;
+              if (F != kBF16) f = ldexpf(f, __ldg(a.xexp + xrow));
+              // weight rows held by this lane: (row g, row g+8) of each m-tile (bf16: sigma(g))
+              const int wr = (F == kBF16) ? sg : g;
+              if (kGateUp) {
+                __nv_bfloat16* o = a.out_routed + (int64_t)xrow * a.N + r0 + warp * 16;
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {
+                  const float gt = acc[q][0][hr * 2 + hc] * f;
+                  const float up = acc[q][1][hr * 2 + hc] * f;
+                  const float h = gt / (1.f + expf(-gt)) * up;
+                  o[wr + 8 * hr] = __float2bfloat16_rn(h);
+                }
+              } else {
+                __nv_bfloat16* o = it.shared_idx >= 0
+                                       ? a.out_shared + ((int64_t)it.shared_idx * a.T + col) * a.N
+                                       : a.out_routed + (int64_t)xrow * a.N;
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                  for (int hr = 0; hr < 2; ++hr)
+                    o[r0 + warp * 32 + mt * 16 + wr + 8 * hr] = __float2bfloat16_rn(acc[q][mt][hr * 2 + hc] * f);
               }
             }
           }
         }
       }
     }
-    if (*s_abort) break;
-    if (Tr::blk) {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sempty[sb]);
+  }
+  if constexpr (Tr::blk != 0) {
+    // every consumer warp is done with tensor memory before warp 0 frees it
+    tc::fence_before_sync();
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+    if (warp == 0) {
+      tc::fence_after_sync();
+      tc::tmem_dealloc(*s_tmem, (uint32_t)a.tmem_alloc);
     }
   }
 }
@@ -538,6 +638,14 @@ static cudaError_t launch_one(const FfnArgs& a, int grid, size_t smem, cudaStrea
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     configured_smem = (int)smem;
+  }
+  if (a.tmem_alloc > 0) {
+    // tcgen05.alloc waits while the SM's 512 columns are taken: never let the
+    // blocks that can share an SM ask for more than that together.
+    int per_sm = 0;
+    cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+    if (err != cudaSuccess) return err;
+    if (per_sm * a.tmem_alloc > 512) return cudaErrorInvalidConfiguration;
   }
   ProfScope prof(GU ? "ffn_stage1_gate_up" : "ffn_stage2_down", st);
   return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, a);
@@ -568,26 +676,42 @@ static int fmt_srow(int F, int K) {
   }
 }
 
-// Shared memory plan of one stage kernel; returns false when it cannot fit.
+// Shared memory plan of one stage kernel: the header, then a ring of stages
+// (weights + activations).  Block scales travel through the same ring, one
+// item's scales in n_sslots stages, so no buffer is set aside for them.
+// Returns false when fewer than two stages fit.
 static bool plan_smem(int F, int ng, int K, int E, int n_shared, int smem_max, FfnArgs& a, size_t& total) {
   const int hdr = stream_hdr_bytes(E, n_shared);
-  const int sbuf = ((kRowsPerStage * fmt_srow(F, K)) + 1023) & ~1023;
   const int stage = kRowsPerStage * kLine + ((fmt_kc(F) * 2) / kLine) * ng * 8 * kLine;
   const int usable = smem_max - 1024;  // room for the runtime 1024-byte alignment
-  for (int nsb = 2; nsb >= 1; --nsb) {
-    const int nsbx = (F == kBF16) ? 1 : nsb;
-    const int room = usable - hdr - nsbx * sbuf;
-    int ns = room / stage;
-    if (ns > kMaxStages) ns = kMaxStages;
-    if (ns >= 3 || (nsb == 1 && ns >= 2)) {
-      a.n_stages = ns;
-      a.n_scale_buf = nsbx;
-      a.smem_scale_bytes = sbuf;
-      total = (size_t)1024 + hdr + (size_t)nsbx * sbuf + (size_t)ns * stage;
-      return true;
-    }
+  int ns = (usable - hdr) / stage;
+  if (ns > kMaxStages) ns = kMaxStages;
+  if (ns < 2) return false;
+  a.n_stages = ns;
+  a.n_sslots = 0;
+  const int srow = fmt_srow(F, K);
+  if (srow > 0) {
+    // each of the 8 consumer warps owns 32 scale rows; split them over 1, 2, 4 or 8 stages
+    int n = 1;
+    while (n < kConsumerWarps && (kConsumerWarps / n) * 32 * srow > stage) n *= 2;
+    if ((kConsumerWarps / n) * 32 * srow > stage) return false;
+    a.n_sslots = n;
   }
-  return false;
+  total = (size_t)1024 + hdr + (size_t)ns * stage;
+  return true;
+}
+
+// TMEM columns for one weight row's block scales: whole 32-bit words, a
+// multiple of 4 (the copy-in stores 4 at a time) and at least every column a
+// K chunk reads.
+static int tmem_scale_cols(int F, int K) {
+  const int srow = fmt_srow(F, K);
+  if (srow == 0) return 0;
+  const int cpc = F == kMXFP4 ? 2 : (F == kNVFP4 ? 4 : 1);
+  int cols = (((srow + 3) / 4) + 3) & ~3;
+  const int need = ceil_div(K, fmt_kc(F)) * cpc;
+  if (cols < need) cols = (need + 3) & ~3;
+  return cols;
 }
 
 cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers& p, int T, int n_sms,
@@ -596,14 +720,23 @@ cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers&
   // Columns per pass (NG groups of 8 activation rows) and CTAs per SM.  Two
   // CTAs of 8 consumer warps hide the decode's fixed-latency dependencies
   // better than one (measured on the gpt-oss decode batch: stage 1 at 4.2 vs
-  // 3.2 TB/s); 16 columns cover almost every routed expert of a decode batch
-  // in one pass.  MOE_FFN_NG / MOE_FFN_MINB override the choice for tuning.
-  int ng = T <= 8 ? 1 : 2;
+  // 3.2 TB/s).  One group of 8 columns covers almost every routed expert of a
+  // decode batch that averages a few rows per expert, and leaves room for the
+  // activation boxes; shared experts (T rows each) and batches that average
+  // four or more rows per expert take 16 columns per pass (measured: Kimi
+  // T=128 1.48 vs 1.67 ms per layer with 16 vs 8, gpt-oss T=64 350 vs 356 us
+  // with 8 vs 16).  Weight boxes keep normal L2 priority: a 128-byte box row
+  // of a 1440-byte weight row straddles 64-byte lines whose other half the
+  // next K chunk reads, and marking them evict-first let L2 drop those halves
+  // before that (DRAM reads 1.125 vs 1.042 GB per stage-1 launch; stage 1
+  // 229 vs 204 us at T=64).  MOE_FFN_NG / MOE_FFN_MINB / MOE_W_L2FIRST
+  // override the choices for tuning.
+  int ng = (T <= 8 || (a.n_shared == 0 && (int64_t)T * a.k < 4LL * a.E)) ? 1 : 2;
   int minb = 2;
   if (const char* e = getenv("MOE_FFN_NG")) ng = atoi(e);
   if (const char* e = getenv("MOE_FFN_MINB")) minb = atoi(e);
   if (ng != 1 && ng != 2 && ng != 4) ng = 2;
-  if (const char* e = getenv("MOE_W_L2NORMAL")) a.w_l2_normal = atoi(e);
+  if (const char* e = getenv("MOE_W_L2FIRST")) a.w_l2_first = atoi(e);
   if (minb == 2 && ng > 2) ng = 2;
   size_t smem = 0;
   bool ok = false;
@@ -615,6 +748,20 @@ cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers&
   if (!ok) {
     *unsupported = 1;
     return cudaSuccess;
+  }
+  // TMEM for the block scales: 2 x tmem_cols columns (two warps per lane
+  // quarter), at most 256 per block so that two co-resident blocks never wait
+  // for each other's columns (launch_one checks the occupancy).
+  a.tmem_cols = tmem_scale_cols(F, a.K);
+  a.tmem_alloc = 0;
+  if (a.tmem_cols > 0) {
+    int alloc = 32;
+    while (alloc < 2 * a.tmem_cols) alloc *= 2;
+    if (alloc > 256) {
+      *unsupported = 1;  // more than 512 scale bytes per weight row
+      return cudaSuccess;
+    }
+    a.tmem_alloc = alloc;
   }
   // tensor maps
   const uint64_t row_bytes = (F == kBF16) ? (uint64_t)a.K * 2 : (uint64_t)a.K / 2;

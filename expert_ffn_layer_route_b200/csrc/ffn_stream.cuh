@@ -30,14 +30,17 @@ struct alignas(64) FfnArgs {
   int K;  // reduction length
   const int32_t* offsets;  // [E+1]
   const int32_t* xexp;     // per activation row power-of-two exponent (4-bit formats)
+  const float* xbias;      // INT4: per activation row and 128-group, the constant part
+                           // 1032 sum(even x) + 1152 sum(odd x') of the offset decode
   // outputs (bf16): stage 1 writes rows [rows_total][d_ff]; stage 2 writes routed
   // rows to out_routed [T*k][d] and shared rows to out_shared [n_shared][T][d]
   __nv_bfloat16* out_routed;
   __nv_bfloat16* out_shared;
   int n_stages;
-  int n_scale_buf;
-  int smem_scale_bytes;  // per buffer
-  int w_l2_normal;       // 1: weight boxes with normal L2 priority, 0: evict-first
+  int n_sslots;    // ring stages that carry one item's block scales (1, 2, 4 or 8)
+  int tmem_cols;   // TMEM columns holding one weight row's block scales
+  int tmem_alloc;  // TMEM columns allocated per block (power of two >= 32)
+  int w_l2_first;        // 1: weight boxes marked evict-first in L2; 0 (default): normal priority
 };
 
 // Launch one stage (gate_up: stage 1 with SwiGLU; else stage 2) of the

@@ -25,7 +25,7 @@ cudaError_t launch_route_topk(const moe_layer_desc& dsc, const void* x, const vo
                               float* logits, int32_t* topk_idx, float* topk_w, cudaStream_t st);
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* offsets, int32_t* row_token,
                            int32_t* inv, cudaStream_t st);
-cudaError_t launch_prep_rows(const void* src, int rows, int K, int mode, void* dst, int32_t* rexp,
+cudaError_t launch_prep_rows(const void* src, int rows, int K, int mode, void* dst, int32_t* rexp, float* gbias,
                              const int32_t* gather, int n_gather, int n_tok, cudaStream_t st);
 cudaError_t launch_combine(const void* y, const int32_t* inv, const float* gw, const void* y_shared, int n_shared,
                            int T, int d, int k, void* out, cudaStream_t st);
@@ -59,7 +59,7 @@ int64_t scale_bytes(int f, int64_t N, int64_t K) {
 }
 
 struct Layout {
-  size_t logits, topk_idx, topk_w, offsets, row_token, inv, xperm, xexp, h, hq, hexp, y, ysh, total;
+  size_t logits, topk_idx, topk_w, offsets, row_token, inv, xperm, xexp, gbias, h, hq, hexp, y, ysh, total;
 };
 
 Layout layout_of(const moe_layer_desc& d) {
@@ -81,6 +81,8 @@ Layout layout_of(const moe_layer_desc& d) {
   const bool q = is4bit(d.wdtype);
   L.xperm = take(RT * D * 2);
   L.xexp = take(q ? RT * 4 : 0);
+  // INT4: per row and 128-wide scale group, stage 1 (K = d) then reused by stage 2 (K = d_ff)
+  L.gbias = take(d.wdtype == MOE_W_INT4_G128 ? RT * ((D > F ? D : F) / 128) * 4 : 0);
   L.h = take(RT * F * 2);
   L.hq = take(q ? RT * F * 2 : 0);
   L.hexp = take(q ? RT * 4 : 0);
@@ -156,9 +158,10 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
   __half* hq = reinterpret_cast<__half*>(ws + L.hq);
   int32_t* hexp = reinterpret_cast<int32_t*>(ws + L.hexp);
+  float* gbias = f == MOE_W_INT4_G128 ? reinterpret_cast<float*>(ws + L.gbias) : nullptr;
   const int mode = !q ? 2 : (f == MOE_W_INT4_G128 ? 1 : 0);
   // activation rows in expert order (routed rows, then every token once per shared expert)
-  err = launch_prep_rows(x, RT, D, mode, xperm, xexp, row_token, R, T, st);
+  err = launch_prep_rows(x, RT, D, mode, xperm, xexp, gbias, row_token, R, T, st);
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   auto fill = [&](FfnArgs& a, FfnPointers& p, bool stage1) {
     std::memset(&a, 0, sizeof(a));
@@ -221,6 +224,7 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
   fill(a1, p1, true);
   p1.x = xperm;
   a1.xexp = q ? xexp : nullptr;
+  a1.xbias = gbias;
   a1.out_routed = h;
   a1.out_shared = nullptr;
   int unsup = 0;
@@ -231,7 +235,7 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
   if (unsup) return MOE_ERR_UNSUPPORTED;
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   if (q) {
-    err = launch_prep_rows(h, RT, F, mode, hq, hexp, nullptr, 0, T, st);
+    err = launch_prep_rows(h, RT, F, mode, hq, hexp, gbias, nullptr, 0, T, st);
     if (err != cudaSuccess) return MOE_ERR_CUDA;
   }
   FfnArgs a2;
@@ -239,6 +243,7 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
   fill(a2, p2, false);
   p2.x = q ? static_cast<const void*>(hq) : static_cast<const void*>(h);
   a2.xexp = q ? hexp : nullptr;
+  a2.xbias = gbias;
   a2.out_routed = static_cast<__nv_bfloat16*>(y_perm);
   a2.out_shared = static_cast<__nv_bfloat16*>(y_shared);
   if (use_gemm)

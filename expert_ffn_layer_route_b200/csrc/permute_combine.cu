@@ -115,15 +115,23 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* off
 // Modes: kCopyBf16 copies the bf16 row; otherwise the row is converted to fp16
 // after scaling by 2^-p with p = floor(log2(max|row|)) - 14, so that its
 // largest magnitude lies in [2^14, 2^15) (fp16's range), and rexp[r] = p is
-// undone on the accumulators.  kPermInt4 stores each 8-element group in the
-// order 0,4,1,5,2,6,3,7, the pairing the INT4 decoder produces.
+// undone on the accumulators.  kF16Int4 serves the INT4 decode, which meets
+// even K with 1024 + (q + 8) and odd K with 1024 + 16 (q + 8): it divides the
+// odd-K values by 16 (a power of two), stores each 8-element group in the
+// order 0,4,1,5,2,6,3,7 (the decoder's pairing), and writes per 128-wide
+// scale group g the constant part of the products,
+//   gbias[r][g] = 1032 * sum_{even k in g} h_k + 1152 * sum_{odd k in g} h_k,
+// over the stored fp16 values h (summed in fp64, rounded once to fp32), so
+// that the grouped FFN recovers sum_k x_k q_k = MMA - gbias exactly up to
+// rounding.
 constexpr int kPrepThreads = 128;
-enum PrepMode : int { kF16 = 0, kF16PermInt4 = 1, kCopyBf16 = 2 };
+enum PrepMode : int { kF16 = 0, kF16Int4 = 1, kCopyBf16 = 2 };
 
 template <int kMode>
 __global__ void __launch_bounds__(kPrepThreads)
     prep_rows_kernel(const __nv_bfloat16* __restrict__ src, int K, void* __restrict__ dst,
-                     int32_t* __restrict__ rexp, const int32_t* __restrict__ gather, int n_gather, int n_tok) {
+                     int32_t* __restrict__ rexp, float* __restrict__ gbias, const int32_t* __restrict__ gather,
+                     int n_gather, int n_tok) {
   pdl_wait_and_trigger();
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
@@ -163,41 +171,59 @@ __global__ void __launch_bounds__(kPrepThreads)
   if (tid == 0) rexp[row] = p;
   const float scale = ldexpf(1.f, -p);
   uint4* d = reinterpret_cast<uint4*>(static_cast<__half*>(dst) + (size_t)row * K);
-  for (int c = tid; c < nchunk; c += kPrepThreads) {
-    const uint4 u = __ldg(s + c);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  // every thread runs the same number of rounds so that the 16-lane group
+  // sums below see full warps (nchunk is a multiple of 16 for INT4)
+  for (int base = 0; base < nchunk; base += kPrepThreads) {
+    const int c = base + tid;
+    const bool on = c < nchunk;
     float f[8];
+    if (on) {
+      const uint4 u = __ldg(s + c);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      f[2 * q] = bf16_bits_to_f32(w[q] & 0xffffu) * scale;
-      f[2 * q + 1] = bf16_bits_to_f32(w[q] >> 16) * scale;
+      for (int q = 0; q < 4; ++q) {
+        f[2 * q] = bf16_bits_to_f32(w[q] & 0xffffu) * scale;
+        f[2 * q + 1] = bf16_bits_to_f32(w[q] >> 16) * scale;
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) f[q] = 0.f;
     }
     __half h[8];
-    if constexpr (kMode == kF16PermInt4) {
+    if constexpr (kMode == kF16Int4) {
       const int order[8] = {0, 4, 1, 5, 2, 6, 3, 7};
+      double even = 0.0, odd = 0.0;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) h[q] = __float2half_rn(f[order[q]]);
+      for (int q = 0; q < 8; ++q) {
+        const int k = order[q];
+        h[q] = __float2half_rn((k & 1) ? f[k] * 0.0625f : f[k]);
+        if (k & 1) odd += (double)__half2float(h[q]); else even += (double)__half2float(h[q]);
+      }
+      double part = 1032.0 * even + 1152.0 * odd;
+#pragma unroll
+      for (int off = 8; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+      if (on && (tid & 15) == 0) gbias[(size_t)row * (K / 128) + (c >> 4)] = (float)part;
     } else {
 #pragma unroll
       for (int q = 0; q < 8; ++q) h[q] = __float2half_rn(f[q]);
     }
-    d[c] = *reinterpret_cast<uint4*>(h);
+    if (on) d[c] = *reinterpret_cast<uint4*>(h);
   }
 }
 
-// mode: 0 fp16 scaled, 1 fp16 scaled in INT4 pairing order, 2 bf16 copy.
-cudaError_t launch_prep_rows(const void* src, int rows, int K, int mode, void* dst, int32_t* rexp,
+// mode: 0 fp16 scaled, 1 fp16 scaled for the INT4 decode (+ gbias), 2 bf16 copy.
+cudaError_t launch_prep_rows(const void* src, int rows, int K, int mode, void* dst, int32_t* rexp, float* gbias,
                              const int32_t* gather, int n_gather, int n_tok, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
   ProfScope prof(gather ? "prep_x_gather" : "prep_h", st);
   const __nv_bfloat16* s = static_cast<const __nv_bfloat16*>(src);
   if (mode == kCopyBf16)
-    return launch_pdl(prep_rows_kernel<kCopyBf16>, dim3(rows), dim3(kPrepThreads), 0, st, s, K, dst, rexp, gather,
-                      n_gather, n_tok);
-  if (mode == kF16PermInt4)
-    return launch_pdl(prep_rows_kernel<kF16PermInt4>, dim3(rows), dim3(kPrepThreads), 0, st, s, K, dst, rexp,
+    return launch_pdl(prep_rows_kernel<kCopyBf16>, dim3(rows), dim3(kPrepThreads), 0, st, s, K, dst, rexp, gbias,
                       gather, n_gather, n_tok);
-  return launch_pdl(prep_rows_kernel<kF16>, dim3(rows), dim3(kPrepThreads), 0, st, s, K, dst, rexp, gather,
+  if (mode == kF16Int4)
+    return launch_pdl(prep_rows_kernel<kF16Int4>, dim3(rows), dim3(kPrepThreads), 0, st, s, K, dst, rexp, gbias,
+                      gather, n_gather, n_tok);
+  return launch_pdl(prep_rows_kernel<kF16>, dim3(rows), dim3(kPrepThreads), 0, st, s, K, dst, rexp, gbias, gather,
                     n_gather, n_tok);
 }
 

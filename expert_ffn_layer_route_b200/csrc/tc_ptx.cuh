@@ -72,5 +72,41 @@ __device__ __forceinline__ void ld_32x32b_x32(uint32_t taddr, uint32_t (&v)[32])
 }
 __device__ __forceinline__ void ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// Four consecutive 32-bit TMEM columns of this thread's lane <- v (warp-wide).
+__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, const uint32_t (&v)[4]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(v[0]), "r"(v[1]),
+               "r"(v[2]), "r"(v[3])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// N (1, 2 or 4) consecutive 32-bit TMEM columns of this thread's lane -> v[0..N).
+// The values are valid only after tmem_ld_wait<N>(v), which names them as
+// operands so that no use can be scheduled before the wait.
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[4]) {
+  if constexpr (N == 1) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v[0]) : "r"(taddr) : "memory");
+  } else if constexpr (N == 2) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=r"(v[0]), "=r"(v[1]) : "r"(taddr)
+                 : "memory");
+  } else {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                 : "r"(taddr)
+                 : "memory");
+  }
+}
+template <int N>
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&v)[4]) {
+  if constexpr (N == 1) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(v[0])::"memory");
+  } else if constexpr (N == 2) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(v[0]), "+r"(v[1])::"memory");
+  } else {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3])::"memory");
+  }
+}
+
 }  // namespace tc
 }  // namespace moe

@@ -45,6 +45,18 @@ def test_layer_matches_oracle(name, shape, T, seed):
     print(f"{name} seed={seed}: rel err {rel:.2e}, ambiguous tokens {n_amb}")
 
 
+def test_int4_offset_decode_with_positive_activations():
+    """The INT4 decode removes, per 128-wide scale group, a constant
+    proportional to the group's activation sum.  All-positive activation rows
+    make that constant largest relative to the result (no cancellation inside
+    the sum), the hardest case for the fp32 accumulation."""
+    shape = mi.KIMI.replace(d_model=896, d_ff=384, n_experts=48)
+    hl = mi.draw_layer(shape, 24, 5)
+    hl["x"] = (hl["x"].float().abs() + 1.0).to(hl["x"].dtype)
+    rel, n_amb = H.full_check(hl, H.run_layer(H.to_device(hl)))
+    print(f"int4 positive activations: rel err {rel:.2e}, ambiguous tokens {n_amb}")
+
+
 @pytest.mark.parametrize("seed", [2])
 def test_tiny_seed2(seed):
     hl, dl = _layer(mi.TINY, 16, seed)
