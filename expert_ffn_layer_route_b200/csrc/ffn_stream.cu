@@ -653,6 +653,7 @@ static cudaError_t launch_one(const FfnArgs& a, int grid, size_t smem, cudaStrea
 
 template <int F, bool GU>
 static cudaError_t dispatch_ng(const FfnArgs& a, int ng, int minb, int grid, size_t smem, cudaStream_t st) {
+  if (minb == 3) return launch_one<F, 1, GU, 3>(a, grid, smem, st);
   if (minb == 2) {
     switch (ng) {
       case 1: return launch_one<F, 1, GU, 2>(a, grid, smem, st);
@@ -732,14 +733,21 @@ cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers&
   // 229 vs 204 us at T=64).  MOE_FFN_NG / MOE_FFN_MINB / MOE_W_L2FIRST
   // override the choices for tuning.
   int ng = (T <= 8 || (a.n_shared == 0 && (int64_t)T * a.k < 4LL * a.E)) ? 1 : 2;
-  int minb = 2;
+  // With one column group a block fits in a third of an SM (two stages of
+  // 36 KB, 72 registers a thread): 24 consumer warps per SM hide more of the
+  // decode's dependency latency than 16 (gpt-oss T=64: stage 1 at 0.77 vs 0.74
+  // of the HBM copy peak; T=8 121 vs 128 us per layer).
+  int minb = ng == 1 ? 3 : 2;
   if (const char* e = getenv("MOE_FFN_NG")) ng = atoi(e);
   if (const char* e = getenv("MOE_FFN_MINB")) minb = atoi(e);
   if (ng != 1 && ng != 2 && ng != 4) ng = 2;
   if (const char* e = getenv("MOE_W_L2FIRST")) a.w_l2_first = atoi(e);
   if (minb == 2 && ng > 2) ng = 2;
+  if (minb == 3 && ng != 1) minb = 2;
   size_t smem = 0;
   bool ok = false;
+  if (minb == 3) ok = plan_smem(F, ng, a.K, a.E, a.n_shared, smem_per_sm / 3 - 1024, a, smem);
+  if (!ok && minb == 3) minb = 2;
   if (minb == 2) ok = plan_smem(F, ng, a.K, a.E, a.n_shared, smem_per_sm / 2 - 1024, a, smem);
   if (!ok) {
     minb = 1;
@@ -760,6 +768,14 @@ cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers&
     if (alloc > 256) {
       *unsupported = 1;  // more than 512 scale bytes per weight row
       return cudaSuccess;
+    }
+    if (minb == 3 && 3 * alloc > 512) {
+      // three blocks per SM would not all get their columns: two per SM
+      minb = 2;
+      if (!plan_smem(F, ng, a.K, a.E, a.n_shared, smem_per_sm / 2 - 1024, a, smem)) {
+        *unsupported = 1;
+        return cudaSuccess;
+      }
     }
     a.tmem_alloc = alloc;
   }
