@@ -27,6 +27,7 @@ CASES = [
     ("tiny", mi.TINY, 16),
     ("mxfp4_gptoss_dims", mi.GPTOSS.replace(n_experts=16), 8),
     ("mxfp4_gptoss_dims_T1", mi.GPTOSS.replace(n_experts=16), 1),
+    ("mxfp4_gptoss_dims_T3", mi.GPTOSS.replace(n_experts=16), 3),
     ("mxfp4_many_rows", mi.GPTOSS.replace(n_experts=4, top_k=2, d_model=576, d_ff=832), 150),
     ("int4_shared", mi.KIMI.replace(d_model=896, d_ff=384, n_experts=48), 40),
     ("int4_shared_T1", mi.KIMI.replace(d_model=896, d_ff=384, n_experts=48), 1),
@@ -73,8 +74,13 @@ def test_stepwise_entry_points_equal_layer_forward():
             assert torch.equal(a[key], b[key]), key
 
 
-def test_deterministic_across_runs():
-    hl, dl = _layer(mi.GPTOSS.replace(n_experts=32), 24, 4)
+@pytest.mark.parametrize("shape,T", [(mi.GPTOSS.replace(n_experts=32), 24),
+                                     (mi.GPTOSS.replace(n_experts=16), 1),
+                                     (mi.KIMI.replace(d_model=896, d_ff=384, n_experts=48), 2)],
+                         ids=["mxfp4_T24", "mxfp4_T1", "int4_T2"])
+def test_deterministic_across_runs(shape, T):
+    """Bit-identical outputs run to run, from single-token batches up."""
+    hl, dl = _layer(shape, T, 4)
     a = H.run_layer(dl)["out"].clone()
     for _ in range(3):
         assert torch.equal(a, H.run_layer(dl)["out"])
