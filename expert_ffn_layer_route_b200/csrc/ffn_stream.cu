@@ -161,7 +161,8 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
   volatile int* s_abort = reinterpret_cast<volatile int*>(empty + kMaxStages);
   int* s_ngroups = reinterpret_cast<int*>(empty + kMaxStages) + 1;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(empty + kMaxStages) + 2;
-  int* s_offs = reinterpret_cast<int*>(empty + kMaxStages) + 4;  // [E+1]
+  volatile int* s_hdr = reinterpret_cast<volatile int*>(empty + kMaxStages) + 4;  // [kMaxStages] item of a stage
+  int* s_offs = reinterpret_cast<int*>(empty + kMaxStages) + 16;                  // [E+1]
   int* s_gitem = s_offs + (a.E + 4);                             // [groups+1]
   int* s_gexp = s_gitem + (a.E + a.n_shared + 4);                // [groups]
   uint8_t* s_stage = smem + stream_hdr_bytes(a.E, a.n_shared);
@@ -242,6 +243,16 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
   const int n_sslots = Tr::blk ? a.n_sslots : 0;  // ring stages carrying an item's block scales
   const int slot_warps = kConsumerWarps / (n_sslots ? n_sslots : 1);
   const int x_row_bytes = K * 2;
+  // Block b starts with item b.  With more than three items per block the
+  // items after the first gridDim.x are claimed one at a time from a
+  // launch-wide counter (zeroed before the launch), so that blocks that run
+  // faster take more of them (Kimi T=128: 1.35 vs 1.41 ms per layer); the
+  // first ring stage of every item then carries its index in s_hdr for the
+  // consumers, and a last stage with index -1 ends the work.  With fewer,
+  // block b takes items b, b + gridDim.x, ... and consumers follow the same
+  // sequence on their own (the claims cost more than the balance gained:
+  // gpt-oss stage 2 at T=64, 2.97 items per block, 114 vs 108 us).
+  const bool dynamic = n_items > 3 * (int)gridDim.x;
 
   if (warp == kConsumerWarps) {
     // ===================================================== producer warp
@@ -252,7 +263,12 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
       const uint64_t pol_w = a.w_l2_first ? l2_evict_first_policy() : l2_evict_normal_policy();
       const uint64_t pol_x = l2_evict_last_policy();
       uint32_t cnt = 0;
-      for (int item = blockIdx.x; item < n_items && !*s_abort; item += gridDim.x) {
+      int item = blockIdx.x;
+      // claim a ring's depth (+1) ahead of the item's end: the answer is back
+      // before the producer needs it, and the claimed item waits only that long
+      const int claim_at = max(0, nchunks - 1 - nstage);
+      while (item < n_items && !*s_abort) {
+        int next_item = n_items;
         const Item it = decode_item<F>(a, item, ntile, s_gitem, s_gexp, ngroups, s_offs);
         const int r0 = it.tile * rows_per_item;
         const int nrows = min(rows_per_item, a.N - r0);
@@ -267,6 +283,7 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
             *s_abort = 1;
             break;
           }
+          s_hdr[s] = item;
           uint8_t* dst = s_stage + s * STAGE_BYTES;
           const int wrows = kGateUp ? 16 : 32;  // scale rows per warp and matrix half
           const int first = j * slot_warps * wrows;
@@ -285,11 +302,13 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
         const int nbox_w = kGateUp ? 2 : (nrows > kBoxRows ? 2 : 1);
         const int c0 = it.pass * XCOLS;
         for (int ch = 0; ch < nchunks && !*s_abort; ++ch) {
+          if (ch == claim_at) next_item = dynamic ? (int)gridDim.x + atomicAdd(a.work_ctr, 1) : item + (int)gridDim.x;
           const int s = cnt % nstage;
           if (!mbar_wait(&empty[s], ((cnt / nstage) & 1u) ^ 1u)) {
             *s_abort = 1;
             break;
           }
+          s_hdr[s] = item;
           uint8_t* st_w = s_stage + s * STAGE_BYTES;
           uint8_t* st_x = st_w + W_BYTES;
           const int kb = ch * kLine;                 // byte offset inside a weight row
@@ -310,6 +329,18 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
               tma_load_2d(st_x + q * XCOLS * kLine, &a.tm_x, xb0 + q * kLine, it.xrow0 + c0, &full[s], pol_x);
           }
           ++cnt;
+        }
+        item = next_item;
+      }
+      // end of work: one more stage whose header says so
+      if (dynamic && !*s_abort) {
+        const int s = cnt % nstage;
+        if (mbar_wait(&empty[s], ((cnt / nstage) & 1u) ^ 1u)) {
+          s_hdr[s] = -1;
+          mbar_arrive(&full[s]);
+          ++cnt;
+        } else {
+          *s_abort = 1;
         }
       }
       // Let every load this lane issued land before the block can exit.
@@ -347,7 +378,21 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
                             : 32 * s_wl + 16 * (c >> 1) + g + 8 * (c & 1);
   uint32_t cnt = 0;
   const uint32_t stage0 = smem_u32(s_stage);
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+  for (int item = blockIdx.x;; item += gridDim.x) {
+    if (dynamic) {
+      // the item's first stage names it (or the end of work); the loops
+      // below wait on it again: that phase is complete and cannot move on
+      // before this warp releases the stage
+      const int s = cnt % nstage;
+      if (*s_abort || !mbar_wait(&full[s], (cnt / nstage) & 1u)) {
+        *s_abort = 1;
+        break;
+      }
+      item = s_hdr[s];
+      if (item < 0) break;
+    } else if (item >= n_items) {
+      break;
+    }
     const Item it = decode_item<F>(a, item, ntile, s_gitem, s_gexp, ngroups, s_offs);
     const int r0 = it.tile * rows_per_item;
     const int nrows = min(rows_per_item, a.N - r0);

@@ -41,6 +41,7 @@ struct alignas(64) FfnArgs {
   int tmem_cols;   // TMEM columns holding one weight row's block scales
   int tmem_alloc;  // TMEM columns allocated per block (power of two >= 32)
   int w_l2_first;        // 1: weight boxes marked evict-first in L2; 0 (default): normal priority
+  int32_t* work_ctr;     // launch-wide item counter, zero before the launch
 };
 
 // Launch one stage (gate_up: stage 1 with SwiGLU; else stage 2) of the

@@ -26,7 +26,8 @@ cudaError_t launch_route_topk(const moe_layer_desc& dsc, const void* x, const vo
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* offsets, int32_t* row_token,
                            int32_t* inv, cudaStream_t st);
 cudaError_t launch_prep_rows(const void* src, int rows, int K, int mode, void* dst, int32_t* rexp, float* gbias,
-                             const int32_t* gather, int n_gather, int n_tok, cudaStream_t st);
+                             const int32_t* gather, int n_gather, int n_tok, int32_t* zero, int n_zero,
+                             cudaStream_t st);
 cudaError_t launch_combine(const void* y, const int32_t* inv, const float* gw, const void* y_shared, int n_shared,
                            int T, int d, int k, void* out, cudaStream_t st);
 
@@ -59,7 +60,7 @@ int64_t scale_bytes(int f, int64_t N, int64_t K) {
 }
 
 struct Layout {
-  size_t logits, topk_idx, topk_w, offsets, row_token, inv, xperm, xexp, gbias, h, hq, hexp, y, ysh, total;
+  size_t logits, topk_idx, topk_w, offsets, row_token, inv, xperm, xexp, gbias, h, hq, hexp, y, ysh, ctr, total;
 };
 
 Layout layout_of(const moe_layer_desc& d) {
@@ -88,6 +89,7 @@ Layout layout_of(const moe_layer_desc& d) {
   L.hexp = take(q ? RT * 4 : 0);
   L.y = take(R * D * 2);
   L.ysh = take(S * T * D * 2);
+  L.ctr = take(2 * 4);  // work counters of the two streaming FFN stages
   L.total = o;
   return L;
 }
@@ -161,7 +163,9 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
   float* gbias = f == MOE_W_INT4_G128 ? reinterpret_cast<float*>(ws + L.gbias) : nullptr;
   const int mode = !q ? 2 : (f == MOE_W_INT4_G128 ? 1 : 0);
   // activation rows in expert order (routed rows, then every token once per shared expert)
-  err = launch_prep_rows(x, RT, D, mode, xperm, xexp, gbias, row_token, R, T, st);
+  // (also zeroes the work counters of both FFN stages)
+  int32_t* ctr = reinterpret_cast<int32_t*>(ws + L.ctr);
+  err = launch_prep_rows(x, RT, D, mode, xperm, xexp, gbias, row_token, R, T, ctr, 2, st);
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   auto fill = [&](FfnArgs& a, FfnPointers& p, bool stage1) {
     std::memset(&a, 0, sizeof(a));
@@ -225,6 +229,7 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
   p1.x = xperm;
   a1.xexp = q ? xexp : nullptr;
   a1.xbias = gbias;
+  a1.work_ctr = ctr;
   a1.out_routed = h;
   a1.out_shared = nullptr;
   int unsup = 0;
@@ -235,7 +240,7 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
   if (unsup) return MOE_ERR_UNSUPPORTED;
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   if (q) {
-    err = launch_prep_rows(h, RT, F, mode, hq, hexp, gbias, nullptr, 0, T, st);
+    err = launch_prep_rows(h, RT, F, mode, hq, hexp, gbias, nullptr, 0, T, nullptr, 0, st);
     if (err != cudaSuccess) return MOE_ERR_CUDA;
   }
   FfnArgs a2;
@@ -244,6 +249,7 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
   p2.x = q ? static_cast<const void*>(hq) : static_cast<const void*>(h);
   a2.xexp = q ? hexp : nullptr;
   a2.xbias = gbias;
+  a2.work_ctr = ctr + 1;
   a2.out_routed = static_cast<__nv_bfloat16*>(y_perm);
   a2.out_shared = static_cast<__nv_bfloat16*>(y_shared);
   if (use_gemm)

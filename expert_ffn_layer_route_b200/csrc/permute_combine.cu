@@ -131,10 +131,11 @@ template <int kMode>
 __global__ void __launch_bounds__(kPrepThreads)
     prep_rows_kernel(const __nv_bfloat16* __restrict__ src, int K, void* __restrict__ dst,
                      int32_t* __restrict__ rexp, float* __restrict__ gbias, const int32_t* __restrict__ gather,
-                     int n_gather, int n_tok) {
+                     int n_gather, int n_tok, int32_t* __restrict__ zero, int n_zero) {
   pdl_wait_and_trigger();
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
+  for (int i = row * kPrepThreads + tid; i < n_zero; i += gridDim.x * kPrepThreads) zero[i] = 0;
   int srow = row;
   if (gather) srow = row < n_gather ? __ldg(gather + row) : (row - n_gather) % n_tok;
   const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)srow * K);
@@ -212,19 +213,21 @@ __global__ void __launch_bounds__(kPrepThreads)
 }
 
 // mode: 0 fp16 scaled, 1 fp16 scaled for the INT4 decode (+ gbias), 2 bf16 copy.
+// zero[0..n_zero) is cleared on the way (counters the next kernels start from).
 cudaError_t launch_prep_rows(const void* src, int rows, int K, int mode, void* dst, int32_t* rexp, float* gbias,
-                             const int32_t* gather, int n_gather, int n_tok, cudaStream_t st) {
+                             const int32_t* gather, int n_gather, int n_tok, int32_t* zero, int n_zero,
+                             cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
   ProfScope prof(gather ? "prep_x_gather" : "prep_h", st);
   const __nv_bfloat16* s = static_cast<const __nv_bfloat16*>(src);
   if (mode == kCopyBf16)
     return launch_pdl(prep_rows_kernel<kCopyBf16>, dim3(rows), dim3(kPrepThreads), 0, st, s, K, dst, rexp, gbias,
-                      gather, n_gather, n_tok);
+                      gather, n_gather, n_tok, zero, n_zero);
   if (mode == kF16Int4)
     return launch_pdl(prep_rows_kernel<kF16Int4>, dim3(rows), dim3(kPrepThreads), 0, st, s, K, dst, rexp, gbias,
-                      gather, n_gather, n_tok);
+                      gather, n_gather, n_tok, zero, n_zero);
   return launch_pdl(prep_rows_kernel<kF16>, dim3(rows), dim3(kPrepThreads), 0, st, s, K, dst, rexp, gbias, gather,
-                    n_gather, n_tok);
+                    n_gather, n_tok, zero, n_zero);
 }
 
 // ---------------------------------------------------------------------------
