@@ -140,13 +140,21 @@ __device__ __forceinline__ Item decode_item(const FfnArgs& a, int item, int ntil
   return it;
 }
 
-template <int F, int NG, bool kGateUp, int MINB>
+template <int F, int NG, bool kGateUp, int MINB, bool kHalf>
 __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid_constant__ FfnArgs a) {
   using Tr = FmtTraits<F>;
   constexpr int KC = Tr::kc;
   constexpr int XCOLS = NG * 8;                 // activation rows per pass
   constexpr int NXBOX = (KC * 2) / kLine;       // 128-byte activation boxes per stage
-  constexpr int W_BYTES = kRowsPerStage * kLine;
+  // Item geometry.  Full items: 128 gate + 128 up rows (stage 1) or 256 rows
+  // (stage 2), two m16 tiles per consumer warp.  Half items (kHalf, for
+  // batches whose items would not fill the grid): 64 + 64 or 128 rows, one
+  // m16 tile per warp -- in stage 1 its rows g are gate rows and its rows g+8
+  // the up rows of the same outputs.
+  constexpr int kMT = kHalf ? 1 : 2;                                             // m16 tiles per warp
+  constexpr int kItemRows = kGateUp ? (kHalf ? 64 : 128) : (kHalf ? 128 : 256);  // output rows per item
+  constexpr int kWarpRows = kItemRows / kConsumerWarps;                          // output rows per warp
+  constexpr int W_BYTES = (kGateUp ? 2 * kItemRows : kItemRows) * kLine;
   constexpr int X_BYTES = NXBOX * XCOLS * kLine;
   constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
   constexpr int kCpc = Tr::kcpc;                // TMEM scale columns per K chunk
@@ -179,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
   pdl_wait_and_trigger();
   for (int i = tid; i <= E; i += kThreads) s_offs[i] = __ldg(a.offsets + i);
   __syncthreads();
-  const int rows_per_item = kGateUp ? kRowsPerStage / 2 : kRowsPerStage;
+  const int rows_per_item = kItemRows;
   const int ntile = ceil_div(a.N, rows_per_item);
   if (warp == 0) {
     // Block scales live in tensor memory while an item runs: lane i of warp w
@@ -285,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
           }
           s_hdr[s] = item;
           uint8_t* dst = s_stage + s * STAGE_BYTES;
-          const int wrows = kGateUp ? 16 : 32;  // scale rows per warp and matrix half
+          const int wrows = kWarpRows;  // scale rows per warp and matrix half
           const int first = j * slot_warps * wrows;
           const int cnt_rows = max(0, min(nrows - first, slot_warps * wrows));
           const uint32_t bytes = (uint32_t)(cnt_rows * srow);
@@ -299,7 +307,8 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
           ++cnt;
         }
         // boxes of weight rows: stage 1 gate rows r0.. and up rows N+r0..; stage 2 rows r0.., r0+128..
-        const int nbox_w = kGateUp ? 2 : (nrows > kBoxRows ? 2 : 1);
+        const int nbox_w = kGateUp ? 2 : (!kHalf && nrows > kBoxRows ? 2 : 1);
+        constexpr int kBoxH = kGateUp ? kItemRows : kBoxRows;  // rows per weight box
         const int c0 = it.pass * XCOLS;
         for (int ch = 0; ch < nchunks && !*s_abort; ++ch) {
           if (ch == claim_at) next_item = dynamic ? (int)gridDim.x + atomicAdd(a.work_ctr, 1) : item + (int)gridDim.x;
@@ -315,12 +324,12 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
           const int xb0 = ch * KC * 2;               // byte offset inside an activation row
           int nxb = 0;
           for (int q = 0; q < NXBOX; ++q) nxb += (xb0 + q * kLine < x_row_bytes) ? 1 : 0;
-          const uint32_t bytes = it.valid ? (uint32_t)(nbox_w * kBoxRows * kLine + nxb * XCOLS * kLine) : 0u;
+          const uint32_t bytes = it.valid ? (uint32_t)(nbox_w * kBoxH * kLine + nxb * XCOLS * kLine) : 0u;
           mbar_arrive_expect_tx(&full[s], bytes);
           if (it.valid) {
             if (kGateUp) {
               tma_load_3d(st_w, tw, kb, r0, it.phys, &full[s], pol_w);
-              tma_load_3d(st_w + kBoxRows * kLine, tw, kb, a.N + r0, it.phys, &full[s], pol_w);
+              tma_load_3d(st_w + kItemRows * kLine, tw, kb, a.N + r0, it.phys, &full[s], pol_w);
             } else {
               tma_load_3d(st_w, tw, kb, r0, it.phys, &full[s], pol_w);
               if (nbox_w == 2) tma_load_3d(st_w + kBoxRows * kLine, tw, kb, r0 + kBoxRows, it.phys, &full[s], pol_w);
@@ -354,8 +363,8 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
   const int g = lane >> 2, c = lane & 3;
   const int sg = sigma8(g);
   // Rows of this warp's two m16 tiles inside a stage (multiples of 16).
-  const int m0 = kGateUp ? warp * 16 : warp * 32;
-  constexpr int kDm = kGateUp ? kRowsPerStage / 2 : 16;  // second m-tile, rows below the first
+  const int m0 = warp * kWarpRows;  // stage 1: this warp's gate rows; stage 2: its first row
+  constexpr int kDm = kGateUp ? kItemRows : 16;  // full items: second m-tile, rows below the first
   // Stage-relative byte offsets of this lane's operands.  A 128-byte row r
   // keeps its 16-byte granule j at ((j ^ (r & 7)) << 4) (TMA 128-byte
   // swizzle).  For every row this lane reads, r & 7 is g (4-bit codes) or
@@ -364,7 +373,8 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
   // m-tile sit at fixed distances from it.
   const uint32_t w_lane = (F == kBF16) ? (uint32_t)(m0 + sg) * kLine + ((uint32_t)(c ^ sg) << 4)
                                        : (uint32_t)(m0 + g) * kLine + ((uint32_t)g << 4) + 4u * c;
-  constexpr uint32_t kRow8 = 8 * kLine;
+  // A-fragment rows g -> g + 8: the next 8 rows, or (half stage 1) the up rows
+  constexpr uint32_t kRow8 = (kGateUp && kHalf) ? kItemRows * kLine : 8 * kLine;
   constexpr uint32_t kDmBytes = kDm * kLine;
   const uint32_t x_lane = W_BYTES + (uint32_t)sg * kLine + ((uint32_t)(c ^ sg) << 4);
   // Block scales: lane c of a quad owns the scale row of m-tile c>>1, row
@@ -374,8 +384,11 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
                                  : 0u;
   // the owned row inside its scale stage (gate rows of the stage's warps, then up rows)
   const int s_wl = warp % slot_warps;
-  const int s_row = kGateUp ? ((c >> 1) ? 16 * slot_warps : 0) + 16 * s_wl + g + 8 * (c & 1)
-                            : 32 * s_wl + 16 * (c >> 1) + g + 8 * (c & 1);
+  // (half items own two rows per quad: lanes c and c+2 hold the same one)
+  const int s_row = kHalf ? (kGateUp ? ((c & 1) ? kWarpRows * slot_warps : 0) + kWarpRows * s_wl + g
+                                     : kWarpRows * s_wl + g + 8 * (c & 1))
+                          : (kGateUp ? ((c >> 1) ? kWarpRows * slot_warps : 0) + kWarpRows * s_wl + g + 8 * (c & 1)
+                                     : kWarpRows * s_wl + 16 * (c >> 1) + g + 8 * (c & 1));
   uint32_t cnt = 0;
   const uint32_t stage0 = smem_u32(s_stage);
   for (int item = blockIdx.x;; item += gridDim.x) {
@@ -396,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
     const Item it = decode_item<F>(a, item, ntile, s_gitem, s_gexp, ngroups, s_offs);
     const int r0 = it.tile * rows_per_item;
     const int nrows = min(rows_per_item, a.N - r0);
-    const bool active = it.valid && (kGateUp ? (warp * 16 < nrows) : (warp * 32 < nrows));
+    const bool active = it.valid && m0 < nrows;
     const int c0 = it.pass * XCOLS;
     const int ncols = min(XCOLS, it.n_cols - c0);
     const int ng_act = ceil_div(ncols, 8);
@@ -432,14 +445,14 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
       ++cnt;
     }
     if (*s_abort) break;
-    float acc[NG][2][4];
+    float acc[NG][kMT][4];
 #pragma unroll
     for (int q = 0; q < NG; ++q)
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
+      for (int mt = 0; mt < kMT; ++mt)
 #pragma unroll
         for (int r = 0; r < 4; ++r) acc[q][mt][r] = 0.f;
-    float tmp[NG][2][4];  // INT4 group partials
+    float tmp[NG][kMT][4];  // INT4 group partials
     float gbias[NG][2];   // INT4 constant part of the group's partials, per column
     const int n_grp = K / 128;
     for (int ch = 0; ch < nchunks; ++ch) {
@@ -475,19 +488,19 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
         auto block = [&](const int b, auto nq_tag, auto guard_tag) {
           constexpr int NQ = decltype(nq_tag)::value;
           constexpr bool kGuard = decltype(guard_tag)::value;
-          [[maybe_unused]] float scb[2][2];  // MXFP4 scale of block b for [m-tile][row g / g+8]
+          [[maybe_unused]] float scb[kMT][2];  // MXFP4 scale of block b for [m-tile][row g / g+8]
           if constexpr (F == kMXFP4) {
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
+            for (int mt = 0; mt < kMT; ++mt)
 #pragma unroll
               for (int hr = 0; hr < 2; ++hr)
                 scb[mt][hr] = __shfl_sync(0xffffffffu, sc8[b], (lane & ~3) | (2 * mt + hr));
           }
-          uint32_t A[2][2][4];  // [m-tile][k16 tile][reg]
+          uint32_t A[kMT][2][4];  // [m-tile][k16 tile][reg]
           if constexpr (F == kBF16) {
             const uint32_t wa = wa0 ^ ((uint32_t)b << 6);
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
+            for (int mt = 0; mt < kMT; ++mt) {
               const uint4 lo = lds128(wa + mt * kDmBytes);
               const uint4 hi = lds128(wa + mt * kDmBytes + kRow8);
               A[mt][0][0] = lo.x; A[mt][0][1] = hi.x; A[mt][0][2] = lo.y; A[mt][0][3] = hi.y;
@@ -498,17 +511,17 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
             // NVFP4: the two 16-block scales of block b of each owned row sit in
             // one 16-bit half of the row's chunk word b>>1; this lane's 8 values
             // lie in 16-block 2b + (c>>1)
-            [[maybe_unused]] uint32_t nv[2][2];
+            [[maybe_unused]] uint32_t nv[kMT][2];
             if constexpr (F == kNVFP4) {
 #pragma unroll
-              for (int mt = 0; mt < 2; ++mt)
+              for (int mt = 0; mt < kMT; ++mt)
 #pragma unroll
                 for (int hr = 0; hr < 2; ++hr)
                   nv[mt][hr] = __shfl_sync(0xffffffffu, sv[b >> 1], (lane & ~3) | (2 * mt + hr)) >>
                                (16 * (b & 1) + 8 * (c >> 1));
             }
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
+            for (int mt = 0; mt < kMT; ++mt) {
               const uint32_t wlo = lds32(wa + mt * kDmBytes);
               const uint32_t whi = lds32(wa + mt * kDmBytes + kRow8);
               uint32_t l0, l1, l2, l3, h0, h1, h2, h3;
@@ -553,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
             if (kGuard && q >= ng_act) break;
             const uint4 xv = lds128(xa + q * 8 * kLine);
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
+            for (int mt = 0; mt < kMT; ++mt) {
               if constexpr (F == kMXFP4) {
                 float t4[4];
                 mma_f16_z(t4, A[mt][0][0], A[mt][0][1], A[mt][0][2], A[mt][0][3], xv.x, xv.y);
@@ -580,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
             if ((b & 3) == 3 || b == nblk - 1) {
               const int gi = b >> 2;  // group inside the chunk: bf16 half gi of the chunk word
 #pragma unroll
-              for (int mt = 0; mt < 2; ++mt) {
+              for (int mt = 0; mt < kMT; ++mt) {
                 const uint32_t wlo = __shfl_sync(0xffffffffu, sv[0], (lane & ~3) | (2 * mt));
                 const uint32_t whi = __shfl_sync(0xffffffffu, sv[0], (lane & ~3) | (2 * mt + 1));
                 const float s_lo = __uint_as_float(gi ? (wlo & 0xffff0000u) : (wlo << 16));
@@ -639,23 +652,30 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
               // weight rows held by this lane: (row g, row g+8) of each m-tile (bf16: sigma(g))
               const int wr = (F == kBF16) ? sg : g;
               if (kGateUp) {
-                __nv_bfloat16* o = a.out_routed + (int64_t)xrow * a.N + r0 + warp * 16;
+                __nv_bfloat16* o = a.out_routed + (int64_t)xrow * a.N + r0 + m0;
+                if constexpr (kHalf) {
+                  // one m-tile: rows g hold the gate, rows g+8 the up projection
+                  const float gt = acc[q][0][hc] * f;
+                  const float up = acc[q][0][2 + hc] * f;
+                  o[wr] = __float2bfloat16_rn(gt / (1.f + expf(-gt)) * up);
+                } else {
 #pragma unroll
-                for (int hr = 0; hr < 2; ++hr) {
-                  const float gt = acc[q][0][hr * 2 + hc] * f;
-                  const float up = acc[q][1][hr * 2 + hc] * f;
-                  const float h = gt / (1.f + expf(-gt)) * up;
-                  o[wr + 8 * hr] = __float2bfloat16_rn(h);
+                  for (int hr = 0; hr < 2; ++hr) {
+                    const float gt = acc[q][0][hr * 2 + hc] * f;
+                    const float up = acc[q][kMT - 1][hr * 2 + hc] * f;
+                    const float h = gt / (1.f + expf(-gt)) * up;
+                    o[wr + 8 * hr] = __float2bfloat16_rn(h);
+                  }
                 }
               } else {
                 __nv_bfloat16* o = it.shared_idx >= 0
                                        ? a.out_shared + ((int64_t)it.shared_idx * a.T + col) * a.N
                                        : a.out_routed + (int64_t)xrow * a.N;
 #pragma unroll
-                for (int mt = 0; mt < 2; ++mt)
+                for (int mt = 0; mt < kMT; ++mt)
 #pragma unroll
                   for (int hr = 0; hr < 2; ++hr)
-                    o[r0 + warp * 32 + mt * 16 + wr + 8 * hr] = __float2bfloat16_rn(acc[q][mt][hr * 2 + hc] * f);
+                    o[r0 + m0 + mt * 16 + wr + 8 * hr] = __float2bfloat16_rn(acc[q][mt][hr * 2 + hc] * f);
               }
             }
           }
@@ -675,9 +695,9 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
 }
 
 // ------------------------------------------------------------------ host side
-template <int F, int NG, bool GU, int MINB>
+template <int F, int NG, bool GU, int MINB, bool HALF>
 static cudaError_t launch_one(const FfnArgs& a, int grid, size_t smem, cudaStream_t st) {
-  auto kern = ffn_stream_kernel<F, NG, GU, MINB>;
+  auto kern = ffn_stream_kernel<F, NG, GU, MINB, HALF>;
   static thread_local int configured_smem = -1;
   if (configured_smem != (int)smem) {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -697,18 +717,23 @@ static cudaError_t launch_one(const FfnArgs& a, int grid, size_t smem, cudaStrea
 }
 
 template <int F, bool GU>
-static cudaError_t dispatch_ng(const FfnArgs& a, int ng, int minb, int grid, size_t smem, cudaStream_t st) {
-  if (minb == 3) return launch_one<F, 1, GU, 3>(a, grid, smem, st);
+static cudaError_t dispatch_ng(const FfnArgs& a, int ng, int minb, bool half, int grid, size_t smem,
+                               cudaStream_t st) {
+  if (half) {  // one column group, two or three blocks per SM
+    if (minb == 3) return launch_one<F, 1, GU, 3, true>(a, grid, smem, st);
+    return launch_one<F, 1, GU, 2, true>(a, grid, smem, st);
+  }
+  if (minb == 3) return launch_one<F, 1, GU, 3, false>(a, grid, smem, st);
   if (minb == 2) {
     switch (ng) {
-      case 1: return launch_one<F, 1, GU, 2>(a, grid, smem, st);
-      default: return launch_one<F, 2, GU, 2>(a, grid, smem, st);
+      case 1: return launch_one<F, 1, GU, 2, false>(a, grid, smem, st);
+      default: return launch_one<F, 2, GU, 2, false>(a, grid, smem, st);
     }
   }
   switch (ng) {
-    case 1: return launch_one<F, 1, GU, 1>(a, grid, smem, st);
-    case 2: return launch_one<F, 2, GU, 1>(a, grid, smem, st);
-    default: return launch_one<F, 4, GU, 1>(a, grid, smem, st);
+    case 1: return launch_one<F, 1, GU, 1, false>(a, grid, smem, st);
+    case 2: return launch_one<F, 2, GU, 1, false>(a, grid, smem, st);
+    default: return launch_one<F, 4, GU, 1, false>(a, grid, smem, st);
   }
 }
 
@@ -726,9 +751,11 @@ static int fmt_srow(int F, int K) {
 // (weights + activations).  Block scales travel through the same ring, one
 // item's scales in n_sslots stages, so no buffer is set aside for them.
 // Returns false when fewer than two stages fit.
-static bool plan_smem(int F, int ng, int K, int E, int n_shared, int smem_max, FfnArgs& a, size_t& total) {
+static bool plan_smem(int F, int ng, int K, int E, int n_shared, int smem_max, bool half, FfnArgs& a,
+                      size_t& total) {
   const int hdr = stream_hdr_bytes(E, n_shared);
-  const int stage = kRowsPerStage * kLine + ((fmt_kc(F) * 2) / kLine) * ng * 8 * kLine;
+  const int wrows = half ? kRowsPerStage / 2 : kRowsPerStage;  // weight rows per stage
+  const int stage = wrows * kLine + ((fmt_kc(F) * 2) / kLine) * ng * 8 * kLine;
   const int usable = smem_max - 1024;  // room for the runtime 1024-byte alignment
   int ns = (usable - hdr) / stage;
   if (ns > kMaxStages) ns = kMaxStages;
@@ -737,10 +764,12 @@ static bool plan_smem(int F, int ng, int K, int E, int n_shared, int smem_max, F
   a.n_sslots = 0;
   const int srow = fmt_srow(F, K);
   if (srow > 0) {
-    // each of the 8 consumer warps owns 32 scale rows; split them over 1, 2, 4 or 8 stages
+    // each of the 8 consumer warps owns 32 scale rows (16 with half items);
+    // split them over 1, 2, 4 or 8 stages
+    const int per_warp = half ? 16 : 32;
     int n = 1;
-    while (n < kConsumerWarps && (kConsumerWarps / n) * 32 * srow > stage) n *= 2;
-    if ((kConsumerWarps / n) * 32 * srow > stage) return false;
+    while (n < kConsumerWarps && (kConsumerWarps / n) * per_warp * srow > stage) n *= 2;
+    if ((kConsumerWarps / n) * per_warp * srow > stage) return false;
     a.n_sslots = n;
   }
   total = (size_t)1024 + hdr + (size_t)ns * stage;
@@ -789,14 +818,28 @@ cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers&
   if (const char* e = getenv("MOE_W_L2FIRST")) a.w_l2_first = atoi(e);
   if (minb == 2 && ng > 2) ng = 2;
   if (minb == 3 && ng != 1) minb = 2;
+  // Half items (128 rows of W_down) in stage 2 when full items would fill
+  // fewer than half of the block slots: twice the blocks stream the same
+  // bytes (gpt-oss T=1: stage 2 19.0 vs 23.0 us).  Measured not to pay in
+  // stage 1 (64 + 64-row items: 24.3 vs 23.0 us) nor with long K rows (Kimi
+  // T=1, 28 chunks per item either way: 133 vs 126 us per layer), where each
+  // block's chain of stage round trips, not its bytes, sets the time.
+  // MOE_FFN_HALF=0/1 overrides (either stage).
+  bool half;
+  {
+    const long full_items = (long)(a.n_shared + (a.E < T * a.k ? a.E : T * a.k)) * ceil_div(a.N, gate_up ? 128 : 256);
+    half = !gate_up && ng == 1 && minb >= 2 && 2 * full_items < (long)n_sms * minb;
+    if (const char* e = getenv("MOE_FFN_HALF")) half = atoi(e) != 0 && ng == 1 && minb >= 2;
+  }
   size_t smem = 0;
   bool ok = false;
-  if (minb == 3) ok = plan_smem(F, ng, a.K, a.E, a.n_shared, smem_per_sm / 3 - 1024, a, smem);
+  if (minb == 3) ok = plan_smem(F, ng, a.K, a.E, a.n_shared, smem_per_sm / 3 - 1024, half, a, smem);
   if (!ok && minb == 3) minb = 2;
-  if (minb == 2) ok = plan_smem(F, ng, a.K, a.E, a.n_shared, smem_per_sm / 2 - 1024, a, smem);
+  if (minb == 2) ok = plan_smem(F, ng, a.K, a.E, a.n_shared, smem_per_sm / 2 - 1024, half, a, smem);
   if (!ok) {
     minb = 1;
-    ok = plan_smem(F, ng, a.K, a.E, a.n_shared, smem_max, a, smem);
+    half = false;
+    ok = plan_smem(F, ng, a.K, a.E, a.n_shared, smem_max, false, a, smem);
   }
   if (!ok) {
     *unsupported = 1;
@@ -817,7 +860,7 @@ cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers&
     if (minb == 3 && 3 * alloc > 512) {
       // three blocks per SM would not all get their columns: two per SM
       minb = 2;
-      if (!plan_smem(F, ng, a.K, a.E, a.n_shared, smem_per_sm / 2 - 1024, a, smem)) {
+      if (!plan_smem(F, ng, a.K, a.E, a.n_shared, smem_per_sm / 2 - 1024, half, a, smem)) {
         *unsupported = 1;
         return cudaSuccess;
       }
@@ -827,10 +870,11 @@ cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers&
   // tensor maps
   const uint64_t row_bytes = (F == kBF16) ? (uint64_t)a.K * 2 : (uint64_t)a.K / 2;
   const uint64_t wrows = gate_up ? 2 * (uint64_t)a.N : (uint64_t)a.N;
+  const uint32_t box_rows = (gate_up && half) ? 64u : (uint32_t)kBoxRows;  // rows per weight box
   {
     const uint64_t dims[3] = {row_bytes, wrows, (uint64_t)a.n_phys};
     const uint64_t strides[2] = {row_bytes, (uint64_t)p.stride_w};
-    const uint32_t box[3] = {kLine, kBoxRows, 1};
+    const uint32_t box[3] = {kLine, box_rows, 1};
     if (!encode_tmap_u8(&a.tm_w, p.w, 3, dims, strides, box, true)) {
       *unsupported = 1;
       return cudaSuccess;
@@ -839,7 +883,7 @@ cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers&
   if (a.n_shared > 0) {
     const uint64_t dims[3] = {row_bytes, wrows, (uint64_t)a.n_shared};
     const uint64_t strides[2] = {row_bytes, (uint64_t)p.stride_w_sh};
-    const uint32_t box[3] = {kLine, kBoxRows, 1};
+    const uint32_t box[3] = {kLine, box_rows, 1};
     if (!encode_tmap_u8(&a.tm_wsh, p.w_sh, 3, dims, strides, box, true)) {
       *unsupported = 1;
       return cudaSuccess;
@@ -856,17 +900,17 @@ cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers&
       return cudaSuccess;
     }
   }
-  const int rows_per_item = gate_up ? kRowsPerStage / 2 : kRowsPerStage;
+  const int rows_per_item = gate_up ? (half ? 64 : 128) : (half ? 128 : 256);
   const int ntile = ceil_div(a.N, rows_per_item);
   const long max_items = (long)(a.n_shared + (a.E < T * a.k ? a.E : T * a.k)) * ntile;
   const long slots = (long)n_sms * minb;
   int grid = (int)(max_items < slots ? max_items : slots);
   if (grid < 1) return cudaSuccess;
   switch (F) {
-    case kBF16: return gate_up ? dispatch_ng<kBF16, true>(a, ng, minb, grid, smem, st) : dispatch_ng<kBF16, false>(a, ng, minb, grid, smem, st);
-    case kMXFP4: return gate_up ? dispatch_ng<kMXFP4, true>(a, ng, minb, grid, smem, st) : dispatch_ng<kMXFP4, false>(a, ng, minb, grid, smem, st);
-    case kNVFP4: return gate_up ? dispatch_ng<kNVFP4, true>(a, ng, minb, grid, smem, st) : dispatch_ng<kNVFP4, false>(a, ng, minb, grid, smem, st);
-    default: return gate_up ? dispatch_ng<kINT4, true>(a, ng, minb, grid, smem, st) : dispatch_ng<kINT4, false>(a, ng, minb, grid, smem, st);
+    case kBF16: return gate_up ? dispatch_ng<kBF16, true>(a, ng, minb, half, grid, smem, st) : dispatch_ng<kBF16, false>(a, ng, minb, half, grid, smem, st);
+    case kMXFP4: return gate_up ? dispatch_ng<kMXFP4, true>(a, ng, minb, half, grid, smem, st) : dispatch_ng<kMXFP4, false>(a, ng, minb, half, grid, smem, st);
+    case kNVFP4: return gate_up ? dispatch_ng<kNVFP4, true>(a, ng, minb, half, grid, smem, st) : dispatch_ng<kNVFP4, false>(a, ng, minb, half, grid, smem, st);
+    default: return gate_up ? dispatch_ng<kINT4, true>(a, ng, minb, half, grid, smem, st) : dispatch_ng<kINT4, false>(a, ng, minb, half, grid, smem, st);
   }
 }
 

@@ -58,6 +58,21 @@ def test_int4_offset_decode_with_positive_activations():
     print(f"int4 positive activations: rel err {rel:.2e}, ambiguous tokens {n_amb}")
 
 
+@pytest.mark.parametrize("half", ["0", "1"])
+def test_half_items_forced_in_both_stages(half, monkeypatch):
+    """The streaming FFN's half-height items (64 + 64 rows in stage 1, 128 in
+    stage 2; by default only stage 2 of small batches uses them) forced on and
+    off for every format, against the oracle."""
+    monkeypatch.setenv("MOE_FFN_HALF", half)
+    for shape, T in [(mi.GPTOSS.replace(n_experts=16), 3),
+                     (mi.KIMI.replace(d_model=896, d_ff=384, n_experts=48), 5),
+                     (mi.BANK.replace(d_model=1024, d_ff=384, n_experts=32), 4),
+                     (mi.TINY.replace(n_experts=16, top_k=2), 6)]:
+        hl, dl = _layer(shape, T, 21)
+        rel, n_amb = H.full_check(hl, H.run_layer(dl))
+        print(f"half={half} {shape.name} T={T}: rel err {rel:.2e}, ambiguous {n_amb}")
+
+
 @pytest.mark.parametrize("seed", [2])
 def test_tiny_seed2(seed):
     hl, dl = _layer(mi.TINY, 16, seed)
