@@ -14,8 +14,10 @@
 //   stage 1: h = silu(x W_gate^T) * (x W_up^T)   (gate and up tiles paired)
 //   stage 2: y = h W_down^T
 //
-// Block = 8 consumer warps + 1 producer warp, two blocks per SM, persistent
-// over the work items.  The producer's elected lane issues TMA tiled loads
+// Block = 8 consumer warps + 1 producer warp, three blocks per SM when a pass
+// takes one group of 8 activation rows (else two), persistent over the work
+// items (dynamically claimed when there are more than three per block).  The
+// producer's elected lane issues TMA tiled loads
 // (128-row x 128-byte boxes, 128-byte swizzle) of the weights and of the
 // expert's activation rows into a ring of shared-memory stages, completing on
 // mbarriers.  Consumers decode the 4-bit codes to fp16 (E2M1 with the
@@ -24,7 +26,9 @@
 // with fp32 accumulation.  Block scales: MXFP4 (E8M0 per 32) and INT4 (bf16
 // per 128) multiply the fp32 partial sums of their block; NVFP4 (E4M3 per 16)
 // multiplies the fp16 weights (exact in fp16) and its fp32 global scale is
-// applied in the epilogue.  Within each 32-wide K block lane c of a quad
+// applied in the epilogue.  An item's block scales cross the stage ring once
+// and stay in tensor memory (TMEM) while the item runs, each consumer lane
+// holding one weight row's.  Within each 32-wide K block lane c of a quad
 // holds K = 8c..8c+7, i.e. the MMA's K order is a fixed permutation of the
 // block, applied identically to both operands.  Activation rows (and bf16
 // weight rows) are read through the row order sigma(g) = (g>>1) | (g&1)<<2
