@@ -124,29 +124,36 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* off
 // over the stored fp16 values h (summed in fp64, rounded once to fp32), so
 // that the grouped FFN recovers sum_k x_k q_k = MMA - gbias exactly up to
 // rounding.
-constexpr int kPrepThreads = 128;
+// One thread per 8-element chunk of a row (rounded up to whole warps, at
+// least 128 and at most 1024): a row's loads are then one round deep.
+constexpr int kRowThreadsMin = 128, kRowThreadsMax = 1024;
+static int row_threads(int K) {
+  int t = ((K / 8 + 31) / 32) * 32;
+  return t < kRowThreadsMin ? kRowThreadsMin : (t > kRowThreadsMax ? kRowThreadsMax : t);
+}
 enum PrepMode : int { kF16 = 0, kF16Int4 = 1, kCopyBf16 = 2 };
 
 template <int kMode>
-__global__ void __launch_bounds__(kPrepThreads)
+__global__ void __launch_bounds__(kRowThreadsMax)
     prep_rows_kernel(const __nv_bfloat16* __restrict__ src, int K, void* __restrict__ dst,
                      int32_t* __restrict__ rexp, float* __restrict__ gbias, const int32_t* __restrict__ gather,
                      int n_gather, int n_tok, int32_t* __restrict__ zero, int n_zero) {
   pdl_wait_and_trigger();
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
-  for (int i = row * kPrepThreads + tid; i < n_zero; i += gridDim.x * kPrepThreads) zero[i] = 0;
+  const int nth = blockDim.x;
+  for (int i = row * nth + tid; i < n_zero; i += gridDim.x * nth) zero[i] = 0;
   int srow = row;
   if (gather) srow = row < n_gather ? __ldg(gather + row) : (row - n_gather) % n_tok;
   const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)srow * K);
   const int nchunk = K / 8;
   if constexpr (kMode == kCopyBf16) {
     uint4* d = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + (size_t)row * K);
-    for (int c = tid; c < nchunk; c += kPrepThreads) d[c] = __ldg(s + c);
+    for (int c = tid; c < nchunk; c += nth) d[c] = __ldg(s + c);
     return;
   }
   float amax = 0.f;
-  for (int c = tid; c < nchunk; c += kPrepThreads) {
+  for (int c = tid; c < nchunk; c += nth) {
     const uint4 u = __ldg(s + c);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -157,12 +164,12 @@ __global__ void __launch_bounds__(kPrepThreads)
   }
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  __shared__ float red[kPrepThreads / 32];
+  __shared__ float red[kRowThreadsMax / 32];
   if ((tid & 31) == 0) red[tid >> 5] = amax;
   __syncthreads();
   amax = red[0];
 #pragma unroll
-  for (int w = 1; w < kPrepThreads / 32; ++w) amax = fmaxf(amax, red[w]);
+  for (int w = 1; w < nth / 32; ++w) amax = fmaxf(amax, red[w]);
   int p = 0;
   if (amax > 0.f && amax <= 3.0e38f) {
     int ex;
@@ -174,7 +181,7 @@ __global__ void __launch_bounds__(kPrepThreads)
   uint4* d = reinterpret_cast<uint4*>(static_cast<__half*>(dst) + (size_t)row * K);
   // every thread runs the same number of rounds so that the 16-lane group
   // sums below see full warps (nchunk is a multiple of 16 for INT4)
-  for (int base = 0; base < nchunk; base += kPrepThreads) {
+  for (int base = 0; base < nchunk; base += nth) {
     const int c = base + tid;
     const bool on = c < nchunk;
     float f[8];
@@ -221,19 +228,18 @@ cudaError_t launch_prep_rows(const void* src, int rows, int K, int mode, void* d
   ProfScope prof(gather ? "prep_x_gather" : "prep_h", st);
   const __nv_bfloat16* s = static_cast<const __nv_bfloat16*>(src);
   if (mode == kCopyBf16)
-    return launch_pdl(prep_rows_kernel<kCopyBf16>, dim3(rows), dim3(kPrepThreads), 0, st, s, K, dst, rexp, gbias,
+    return launch_pdl(prep_rows_kernel<kCopyBf16>, dim3(rows), dim3(row_threads(K)), 0, st, s, K, dst, rexp, gbias,
                       gather, n_gather, n_tok, zero, n_zero);
   if (mode == kF16Int4)
-    return launch_pdl(prep_rows_kernel<kF16Int4>, dim3(rows), dim3(kPrepThreads), 0, st, s, K, dst, rexp, gbias,
+    return launch_pdl(prep_rows_kernel<kF16Int4>, dim3(rows), dim3(row_threads(K)), 0, st, s, K, dst, rexp, gbias,
                       gather, n_gather, n_tok, zero, n_zero);
-  return launch_pdl(prep_rows_kernel<kF16>, dim3(rows), dim3(kPrepThreads), 0, st, s, K, dst, rexp, gbias, gather,
+  return launch_pdl(prep_rows_kernel<kF16>, dim3(rows), dim3(row_threads(K)), 0, st, s, K, dst, rexp, gbias, gather,
                     n_gather, n_tok, zero, n_zero);
 }
 
 // ---------------------------------------------------------------------------
-constexpr int kCombineThreads = 128;
 
-__global__ void __launch_bounds__(kCombineThreads)
+__global__ void __launch_bounds__(kRowThreadsMax)
     combine_kernel(const __nv_bfloat16* __restrict__ y, const int32_t* __restrict__ inv,
                    const float* __restrict__ gw, const __nv_bfloat16* __restrict__ y_shared, int n_shared, int T,
                    int d, int k, __nv_bfloat16* __restrict__ out) {
@@ -241,7 +247,7 @@ __global__ void __launch_bounds__(kCombineThreads)
   const int t = blockIdx.x;
   const int nchunk = d / 8;
   const int nrows = T * k;
-  for (int c = threadIdx.x; c < nchunk; c += kCombineThreads) {
+  for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
     float acc[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;
@@ -280,7 +286,7 @@ cudaError_t launch_combine(const void* y, const int32_t* inv, const float* gw, c
                            int T, int d, int k, void* out, cudaStream_t st) {
   if (T <= 0) return cudaSuccess;
   ProfScope prof("combine", st);
-  return launch_pdl(combine_kernel, dim3(T), dim3(kCombineThreads), 0, st, static_cast<const __nv_bfloat16*>(y), inv,
+  return launch_pdl(combine_kernel, dim3(T), dim3(row_threads(d)), 0, st, static_cast<const __nv_bfloat16*>(y), inv,
                     gw, static_cast<const __nv_bfloat16*>(y_shared), n_shared, T, d, k,
                     static_cast<__nv_bfloat16*>(out));
 }
