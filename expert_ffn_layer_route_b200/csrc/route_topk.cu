@@ -9,7 +9,7 @@
 // renormalised over the selection.
 //
 // Kernel 1 (router_logits_kernel): a block computes an 8-token x 4-expert tile
-// of logits.  Thread t of 256 owns the 8-element chunks t, t+256, ... of the
+// of logits (1, 2 or 4 tokens when the batch is smaller).  Thread t of 256 owns the 8-element chunks t, t+256, ... of the
 // hidden dimension, accumulates its products in fp32 in that order, then the
 // partial sums are folded by a warp butterfly and the 8 warps are added in a
 // fixed order.  Every logit - every expert column - goes through the same
@@ -26,11 +26,10 @@
 
 namespace moe {
 
-constexpr int kRouterTokens = 8;   // tokens per block
 constexpr int kRouterExperts = 4;  // experts per block
 constexpr int kRouterThreads = 256;
 
-template <bool kFp32Router>
+template <bool kFp32Router, int kRouterTokens>
 __global__ void __launch_bounds__(kRouterThreads)
     router_logits_kernel(const __nv_bfloat16* __restrict__ x, const void* __restrict__ wr,
                          const float* __restrict__ bias, float* __restrict__ logits, int T, int d, int E) {
@@ -169,16 +168,22 @@ __global__ void __launch_bounds__(256)
 cudaError_t launch_route_topk(const moe_layer_desc& dsc, const void* x, const void* wr, const float* bias,
                               float* logits, int32_t* topk_idx, float* topk_w, cudaStream_t st) {
   const int T = dsc.T, d = dsc.d_model, E = dsc.n_experts, k = dsc.top_k;
-  dim3 grid(ceil_div(T, kRouterTokens), ceil_div(E, kRouterExperts));
   {
+  // tokens per block: 8, or the batch rounded up to a power of two when
+  // smaller (a block's thread keeps the same summation order either way)
+  const int tok = T >= 8 ? 8 : (T > 2 ? 4 : T);
+  auto go = [&](auto kern) {
+    return launch_pdl(kern, dim3(ceil_div(T, tok), ceil_div(E, kRouterExperts)), dim3(kRouterThreads), 0, st,
+                      static_cast<const __nv_bfloat16*>(x), wr, bias, logits, T, d, E);
+  };
   ProfScope prof("router_logits", st);
   cudaError_t err;
   if (dsc.router_fp32)
-    err = launch_pdl(router_logits_kernel<true>, grid, dim3(kRouterThreads), 0, st,
-                     static_cast<const __nv_bfloat16*>(x), wr, bias, logits, T, d, E);
+    err = tok == 1 ? go(router_logits_kernel<true, 1>) : tok == 2 ? go(router_logits_kernel<true, 2>)
+        : tok == 4 ? go(router_logits_kernel<true, 4>) : go(router_logits_kernel<true, 8>);
   else
-    err = launch_pdl(router_logits_kernel<false>, grid, dim3(kRouterThreads), 0, st,
-                     static_cast<const __nv_bfloat16*>(x), wr, bias, logits, T, d, E);
+    err = tok == 1 ? go(router_logits_kernel<false, 1>) : tok == 2 ? go(router_logits_kernel<false, 2>)
+        : tok == 4 ? go(router_logits_kernel<false, 4>) : go(router_logits_kernel<false, 8>);
   if (err != cudaSuccess) return err;
   }
   cudaError_t err = cudaGetLastError();
