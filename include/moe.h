@@ -35,8 +35,14 @@
  * Conventions (all entry points):
  *  - Ownership: the caller owns every device buffer and the stream.  No entry
  *    point of the layer path allocates memory; scratch comes from the caller's
- *    `workspace` (size from moe_workspace_size).  The expert cache owns what
+ *    `workspace` (size from moe_workspace_size).  The workspace needs no
+ *    initialisation and holds nothing between calls: the counters a call uses
+ *    are zeroed by that call's own kernels.  The expert cache owns what
  *    moe_cache_init allocates.
+ *  - On-chip resources: while they run, the blocks of the 4-bit streaming FFN
+ *    kernels each hold up to 256 columns of an SM's tensor memory (TMEM) for
+ *    their block scales; a kernel of another library that holds all 512
+ *    columns of an SM delays them until it finishes.
  *  - Execution: every compute call enqueues work on `stream` and returns; host
  *    argument checks return synchronously (MOE_ERR_INVALID_ARG /
  *    MOE_ERR_UNSUPPORTED) before anything is enqueued.  Launch failures return
@@ -54,12 +60,17 @@
  *      BF16  : plain bf16 values, no scales.
  *  - Shapes: d_model and d_ff must be multiples of 32 (of 128 for INT4);
  *    1 <= top_k <= min(n_experts, 32); n_experts <= 1024; T >= 0 (T = 0 is a
- *    no-op that returns MOE_OK).
+ *    no-op that returns MOE_OK).  The 4-bit streaming FFN keeps at most 512
+ *    scale bytes per weight row in tensor memory: a reduction length beyond
+ *    16384 (MXFP4), 8192 (NVFP4) or 32768 (INT4) returns MOE_ERR_UNSUPPORTED.
  *  - Numerics: activations bf16, products accumulated in fp32.  The 4-bit paths
  *    feed the tensor cores fp16 operands: E2M1 codes convert to fp16 exactly,
  *    and each activation row is scaled by a power of two so that it fits fp16
  *    (exact for every value of magnitude at least 2^-31 times its row's
- *    largest); the power of two is undone on the fp32 accumulator.
+ *    largest); the power of two is undone on the fp32 accumulator.  INT4 codes
+ *    enter as the exact fp16 integers 1024 + 16^j (q + 8) against activations
+ *    pre-divided by 16 where j = 1, and the constant part of each 128-group
+ *    is subtracted from the fp32 group sum before the group scale.
  *  - Thread safety: calls on different streams with different workspaces may
  *    run concurrently; an expert cache object is not thread-safe.
  */
