@@ -36,8 +36,12 @@ __global__ void __launch_bounds__(kPermThreads)
   pdl_wait_and_trigger();
   for (int e = tid; e < E; e += kPermThreads) counts[e] = 0;
   __syncthreads();
+  // (a batch that fits one tile keeps its indices in shared memory for the
+  // scatter below, which then reads no global memory)
+  const bool one_tile = n <= kPermTile;
   for (int i = tid; i < n; i += kPermThreads) {
     const int e = __ldg(idx + i);
+    if (one_tile) tile[i] = e;
     if (e < 0 || e >= E) {
       set_status(MOE_ERR_DEVICE_INDEX);
       inv[i] = -1;
@@ -76,8 +80,10 @@ __global__ void __launch_bounds__(kPermThreads)
   __syncthreads();
   for (int base = 0; base < n; base += kPermTile) {
     const int tn = min(kPermTile, n - base);
-    for (int i = tid; i < tn; i += kPermThreads) tile[i] = __ldg(idx + base + i);
-    __syncthreads();
+    if (!one_tile) {
+      for (int i = tid; i < tn; i += kPermThreads) tile[i] = __ldg(idx + base + i);
+      __syncthreads();
+    }
     for (int e = warp; e < E; e += kPermThreads / 32) {
       int run = cursor[e];
       for (int c0 = 0; c0 < tn; c0 += 32) {
