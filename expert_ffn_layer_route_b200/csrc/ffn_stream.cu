@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
   if (warp == 0) {
     // Block scales live in tensor memory while an item runs: lane i of warp w
     // keeps the scales of one weight row in TMEM lane 32 (w % 4) + i, columns
-    // [(w / 4) C, (w / 4 + 1) C).  Two blocks per SM use at most 2 x 256 columns.
+    // [(w / 4) C, (w / 4 + 1) C); an SM's blocks together take <= 512 columns.
     if (Tr::blk) {
       tc::tmem_alloc(s_tmem, (uint32_t)a.tmem_alloc);
       tc::tmem_relinquish();
@@ -287,8 +287,8 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
         const CUtensorMap* tw = it.shared_idx >= 0 ? &a.tm_wsh : &a.tm_w;
         // The item's block scales first, in n_sslots ring stages: stage j holds
         // the rows of consumer warps [j * slot_warps, (j + 1) * slot_warps) --
-        // gate rows then up rows (stage 1), or 32 rows per warp (stage 2) --
-        // each a contiguous range of the row-major scale matrix.
+        // gate rows then up rows (stage 1), or kWarpRows rows per warp (stage 2)
+        // -- each a contiguous range of the row-major scale matrix.
         for (int j = 0; j < n_sslots && !*s_abort; ++j) {
           const int s = cnt % nstage;
           if (!mbar_wait(&empty[s], ((cnt / nstage) & 1u) ^ 1u)) {
@@ -366,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
   // ======================================================= consumer warps
   const int g = lane >> 2, c = lane & 3;
   const int sg = sigma8(g);
-  // Rows of this warp's two m16 tiles inside a stage (multiples of 16).
+  // Rows of this warp's m16 tile(s) inside a stage (multiples of 8).
   const int m0 = warp * kWarpRows;  // stage 1: this warp's gate rows; stage 2: its first row
   constexpr int kDm = kGateUp ? kItemRows : 16;  // full items: second m-tile, rows below the first
   // Stage-relative byte offsets of this lane's operands.  A 128-byte row r
