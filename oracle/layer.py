@@ -77,6 +77,22 @@ def logit_error_bound(x: np.ndarray, wr: np.ndarray, bias: Optional[np.ndarray],
     return gamma(chain + 2) * mag.max(axis=1)
 
 
+def renormalised_softmax(lt: np.ndarray, sel) -> np.ndarray:
+    """Gates of the selected experts ``sel`` (in that order) for one token's
+    logits ``lt``: the softmax over all E logits, renormalised over ``sel``.
+
+    Both steps run on log-probabilities, log p = l - logsumexp(l), so that a
+    selection lying far below the largest logit (a forced one) does not
+    underflow to 0/0; the renormalisation then divides exp(log p_j - c) by its
+    sum over the selection, c the selection's largest log-probability.
+    """
+    m = lt.max()
+    logp = lt - (m + np.log(np.exp(lt - m).sum()))  # log-softmax over all E
+    ls = logp[np.asarray(sel, dtype=np.int64)]
+    q = np.exp(ls - ls.max())
+    return q / q.sum()
+
+
 def topk_select(logits: np.ndarray, k: int):
     """Per token: the k largest logits, descending, the lower index winning ties.
 
@@ -93,9 +109,7 @@ def topk_select(logits: np.ndarray, k: int):
         order = np.lexsort((experts, -lt))  # primary: logit descending; then index ascending
         sel = order[:k]
         idx[t] = sel
-        p = np.exp(lt - lt.max())
-        p = p / p.sum()
-        gates[t] = p[sel] / p[sel].sum()
+        gates[t] = renormalised_softmax(lt, sel)
         if k < E:
             margin[t] = lt[order[k - 1]] - lt[order[k]]
     return idx, gates, margin
@@ -106,9 +120,7 @@ def gates_for(logits: np.ndarray, idx: np.ndarray) -> np.ndarray:
     T = logits.shape[0]
     g = np.zeros(idx.shape, dtype=np.float64)
     for t in range(T):
-        p = np.exp(logits[t] - logits[t].max())
-        p = p / p.sum()
-        g[t] = p[idx[t]] / p[idx[t]].sum()
+        g[t] = renormalised_softmax(logits[t], idx[t])
     return g
 
 
@@ -204,5 +216,5 @@ def dense_expert_outputs(lay: Dict[str, object], e: int, shared: bool = False) -
     return swiglu_ffn(to_f64(lay["x"]), w13, w2)
 
 
-__all__ = ["router_logits", "logit_error_bound", "topk_select", "gates_for", "permute",
+__all__ = ["router_logits", "logit_error_bound", "renormalised_softmax", "topk_select", "gates_for", "permute",
            "silu", "swiglu_ffn", "moe_layer", "dense_expert_outputs", "to_f64", "dequant"]

@@ -5,7 +5,9 @@ that share nothing with it:
 
 * a hand-worked 3-expert layer whose output is a closed form in e;
 * top-k against brute force over every k-subset (with ties);
-* gates against scipy's softmax over the selected logits;
+* gates against scipy's softmax over the selected logits, for the top-k and
+  for forced selections (any subset, any order), plus a forced selection of the
+  worked layer in closed form;
 * the permutation against numpy's stable argsort;
 * k = E with a zero router, E = 1, identical experts and a shared expert
   against a dense SwiGLU MLP written with torch.nn.functional in float64;
@@ -13,7 +15,9 @@ that share nothing with it:
 
 The planted-mistake tests at the end show that each pin rejects a plausible
 slip in the oracle (gate/up swapped, renormalisation dropped, tie rule
-reversed, wrong permutation order, shared expert dropped).
+reversed, wrong permutation order, shared expert dropped; for forced
+selections: renormalisation dropped, the wrong token's logits, sorted instead
+of the given order, the selection or its gates ignored).
 """
 import itertools
 import math
@@ -103,6 +107,63 @@ def pin_topk(topk_fn):
 
 def test_topk_matches_brute_force_and_softmax():
     assert pin_topk(L.topk_select)
+
+
+def pin_gates_for(gates_fn):
+    """Gates of a given (forced) selection: the softmax of the selected logits
+    (scipy), in the selection's own order, for selections that are not the
+    top-k (any k-subset, any order, ties included), on logits large enough
+    that a missing max-shift would overflow."""
+    rng = np.random.default_rng(11)
+    for trial in range(200):
+        T = int(rng.integers(1, 6))
+        E = int(rng.integers(1, 9))
+        k = int(rng.integers(1, E + 1))
+        logits = rng.integers(-3, 4, size=(T, E)).astype(np.float64)
+        if trial % 3 == 0:
+            logits = logits * 300.0  # exp overflows without the shift
+        idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+        g = gates_fn(logits, idx)
+        for t in range(T):
+            ref = scipy.special.softmax(logits[t, idx[t]])
+            if not np.allclose(g[t], ref, rtol=1e-13, atol=1e-15):
+                return False
+            if abs(g[t].sum() - 1.0) > 1e-12:
+                return False
+    return True
+
+
+def test_gates_for_forced_selection_matches_softmax():
+    assert pin_gates_for(L.gates_for)
+
+
+def pin_forced_worked_example(layer_fn):
+    """The worked 3-expert layer with its selection forced to (2, 0), which is
+    not the top-2 (that is (2, 1)): gates = softmax(l2, l0) = softmax(3, 1) in
+    that order; expert 0 has zero weights, so out = g2 * y2 with
+    y2 = (2 h2, 0), h2 = 3 silu(2)."""
+    g2 = 1.0 / (1.0 + math.exp(-2.0))
+    h2 = 3.0 * (2.0 / (1.0 + math.exp(-2.0)))
+    r = layer_fn(_tiny_layer(), forced_idx=np.array([[2, 0]], np.int32))
+    return (r["idx"].tolist() == [[2, 0]] and np.allclose(r["gates"], [[g2, 1.0 - g2]], rtol=0, atol=1e-15)
+            and np.allclose(r["out"], [[g2 * 2.0 * h2, 0.0]], rtol=1e-14, atol=1e-15)
+            and r["inv"].tolist() == [1, 0] and r["counts"].tolist() == [1, 0, 1])
+
+
+def test_forced_selection_worked_example_closed_form():
+    assert pin_forced_worked_example(L.moe_layer)
+
+
+def test_forced_selection_token_subset():
+    """Forced routing with a token subset takes each listed token's own row."""
+    lay = _small("mxfp4", E=8, k=2, d=64, f=64, T=9)
+    rng = np.random.default_rng(3)
+    forced = np.stack([rng.permutation(8)[:2] for _ in range(9)]).astype(np.int32)
+    full = L.moe_layer(lay, forced_idx=forced)
+    sub = L.moe_layer(lay, forced_idx=forced, tokens=[7, 2, 4])
+    assert np.array_equal(sub["idx"], forced[[7, 2, 4]])
+    assert np.allclose(sub["gates"], full["gates"][[7, 2, 4]], rtol=1e-15, atol=0)
+    assert np.allclose(sub["out"], full["out"][[7, 2, 4]], rtol=1e-13, atol=1e-13 * np.abs(full["out"]).max())
 
 
 def test_margin_definition():
@@ -310,6 +371,37 @@ def test_pins_reject_planted_mistakes(monkeypatch):
         r["out"] = r["out"] * lay["shape"].top_k
         return r
     assert not pin_uniform_average(ungated)
+
+    # forced-selection gates without the renormalisation (softmax over all E)
+    def forced_no_renorm(logits, idx):
+        p = scipy.special.softmax(logits, axis=1)
+        return np.take_along_axis(p, idx.astype(np.int64), 1)
+    assert not pin_gates_for(forced_no_renorm)
+
+    # forced-selection gates taken from the wrong token's logits
+    def forced_wrong_token(logits, idx):
+        return L.gates_for(np.roll(logits, 1, axis=0), idx)
+    assert not pin_gates_for(forced_wrong_token)
+
+    # forced-selection gates in sorted instead of the selection's order
+    def forced_sorted(logits, idx):
+        return L.gates_for(logits, np.sort(idx, axis=1))
+    assert not pin_gates_for(forced_sorted)
+
+    # the layer ignoring a forced selection (keeps its own top-k)
+    def ignores_forced(lay, forced_idx=None, **kw):
+        return L.moe_layer(lay, **kw)
+    assert not pin_forced_worked_example(ignores_forced)
+
+    # the layer forcing the selection but keeping the top-k gates
+    orig_gates_for = L.gates_for
+
+    def stale_gates(logits, idx):
+        return L.topk_select(logits, idx.shape[1])[1]
+    with monkeypatch.context() as m:
+        m.setattr(L, "gates_for", stale_gates)
+        assert not pin_forced_worked_example(L.moe_layer)
+    assert L.gates_for is orig_gates_for
 
 
 _orig_topk = L.topk_select
