@@ -69,7 +69,7 @@ _SIGS = {
     "moe_workspace_layout_of": [_DP, ctypes.POINTER(WorkspaceLayout)],
     "moe_route_topk": [_DP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "moe_route_topk_noalloc": [_DP, _P, _P, _P, _P, _P, _P],
-    "moe_permute": [_DP, _P, _P, _P, _P, _P],
+    "moe_permute": [_DP, _P, _P, _P, _P, _P, _P, _P],
     "moe_grouped_ffn": [_DP, _WP, _WP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "moe_combine": [_DP, _P, _P, _P, _P, _P, _P],
     "moe_layer_forward": [_DP, _P, _P, _P, _WP, _WP, _P, _P, ctypes.c_size_t, _P],
@@ -188,9 +188,10 @@ def moe_route_topk_noalloc(desc, x, w_router, logit_bias, topk_idx, topk_w, stre
                                         _ptr(topk_idx), _ptr(topk_w), _stream(stream)), "moe_route_topk_noalloc")
 
 
-def moe_permute(desc, topk_idx, offsets, row_token, inv, stream=None):
-    _check(lib().moe_permute(ctypes.byref(desc), _ptr(topk_idx), _ptr(offsets), _ptr(row_token), _ptr(inv),
-                             _stream(stream)), "moe_permute")
+def moe_permute(desc, topk_idx, offsets, row_token, inv, stream=None, x=None, x_perm=None):
+    """Grouping; with ``x`` also gathers x_perm[r] = x[row_token[r]]."""
+    _check(lib().moe_permute(ctypes.byref(desc), _ptr(topk_idx), _ptr(x), _ptr(offsets), _ptr(row_token),
+                             _ptr(inv), _ptr(x_perm), _stream(stream)), "moe_permute")
 
 
 def moe_grouped_ffn(desc, routed: Weights, shared: Optional[Weights], offsets, row_token, x, y_perm, y_shared,

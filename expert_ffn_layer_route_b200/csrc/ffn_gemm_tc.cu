@@ -344,11 +344,9 @@ bool gemm_path_supported(int F, int N, int K, bool gate_up) {
 template <bool GU>
 static cudaError_t launch_gemm(const GemmArgs& a, int grid, size_t smem, cudaStream_t st) {
   auto kern = ffn_gemm_tc_kernel<GU>;
-  static thread_local int configured = -1;
-  if (configured != (int)smem) {
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  {
+    cudaError_t err = set_dyn_smem_once<ffn_gemm_tc_kernel<GU>>(smem);
     if (err != cudaSuccess) return err;
-    configured = (int)smem;
   }
   ProfScope prof(GU ? "ffn_gemm_stage1_gate_up" : "ffn_gemm_stage2_down", st);
   return launch_pdl(kern, dim3(grid), dim3(kThreadsTc), smem, st, a);

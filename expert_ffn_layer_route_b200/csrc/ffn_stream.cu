@@ -702,11 +702,9 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
 template <int F, int NG, bool GU, int MINB, bool HALF>
 static cudaError_t launch_one(const FfnArgs& a, int grid, size_t smem, cudaStream_t st) {
   auto kern = ffn_stream_kernel<F, NG, GU, MINB, HALF>;
-  static thread_local int configured_smem = -1;
-  if (configured_smem != (int)smem) {
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  {
+    cudaError_t err = set_dyn_smem_once<ffn_stream_kernel<F, NG, GU, MINB, HALF>>(smem);
     if (err != cudaSuccess) return err;
-    configured_smem = (int)smem;
   }
   if (a.tmem_alloc > 0) {
     // tcgen05.alloc waits while the SM's 512 columns are taken: never let the

@@ -300,14 +300,20 @@ moe_status moe_route_topk(const moe_layer_desc* desc, const void* x, const void*
                                      static_cast<cudaStream_t>(stream)));
 }
 
-moe_status moe_permute(const moe_layer_desc* desc, const int32_t* topk_idx, int32_t* offsets, int32_t* row_token,
-                       int32_t* inv, void* stream) {
+moe_status moe_permute(const moe_layer_desc* desc, const int32_t* topk_idx, const void* x, int32_t* offsets,
+                       int32_t* row_token, int32_t* inv, void* x_perm, void* stream) {
   moe_status s = check_desc(desc);
   if (s != MOE_OK) return s;
   if (!offsets) return MOE_ERR_INVALID_ARG;
   if (desc->T > 0 && (!topk_idx || !row_token || !inv)) return MOE_ERR_INVALID_ARG;
-  return from_cuda(launch_permute(topk_idx, desc->T, desc->top_k, desc->n_experts, offsets, row_token, inv,
-                                  static_cast<cudaStream_t>(stream)));
+  if (x && desc->T > 0 && (!x_perm || !aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t err = launch_permute(topk_idx, desc->T, desc->top_k, desc->n_experts, offsets, row_token, inv, st);
+  if (err != cudaSuccess || !x || desc->T == 0) return from_cuda(err);
+  // x_perm[r] = x[row_token[r]] (bf16 rows in expert order)
+  const int R = desc->T * desc->top_k;
+  return from_cuda(launch_prep_rows(x, R, desc->d_model, 2, x_perm, nullptr, nullptr, row_token, R, desc->T,
+                                    nullptr, 0, st));
 }
 
 moe_status moe_grouped_ffn(const moe_layer_desc* desc, const moe_weights* routed, const moe_weights* shared,

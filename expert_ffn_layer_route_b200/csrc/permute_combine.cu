@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(kPermThreads)
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* offsets, int32_t* row_token,
                            int32_t* inv, cudaStream_t st) {
   const size_t smem = (size_t)(2 * E + kPermTile) * sizeof(int);
-  cudaError_t err = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t err = set_dyn_smem_once<permute_kernel>(smem);
   if (err != cudaSuccess) return err;
   ProfScope prof("permute", st);
   return launch_pdl(permute_kernel, dim3(1), dim3(kPermThreads), smem, st, idx, T * k, k, E, offsets, row_token,
@@ -151,16 +151,20 @@ __global__ void __launch_bounds__(kRowThreadsMax)
   for (int i = row * nth + tid; i < n_zero; i += gridDim.x * nth) zero[i] = 0;
   int srow = row;
   if (gather) srow = row < n_gather ? __ldg(gather + row) : (row - n_gather) % n_tok;
-  const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)srow * K);
+  // a gathered row past the grouped rows (a pair the permutation dropped)
+  // has no source: it is written as zeros
+  const bool have = !gather || (unsigned)srow < (unsigned)n_tok;
+  const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)(have ? srow : 0) * K);
+  const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
   const int nchunk = K / 8;
   if constexpr (kMode == kCopyBf16) {
     uint4* d = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + (size_t)row * K);
-    for (int c = tid; c < nchunk; c += nth) d[c] = __ldg(s + c);
+    for (int c = tid; c < nchunk; c += nth) d[c] = have ? __ldg(s + c) : z4;
     return;
   }
   float amax = 0.f;
   for (int c = tid; c < nchunk; c += nth) {
-    const uint4 u = __ldg(s + c);
+    const uint4 u = have ? __ldg(s + c) : z4;
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -192,7 +196,7 @@ __global__ void __launch_bounds__(kRowThreadsMax)
     const bool on = c < nchunk;
     float f[8];
     if (on) {
-      const uint4 u = __ldg(s + c);
+      const uint4 u = have ? __ldg(s + c) : z4;
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {

@@ -207,19 +207,25 @@ cudaError_t launch_route_topk(const moe_layer_desc& dsc, const void* x, const vo
 //
 // Host code must not pass the array's name to a kernel: on the host it is a
 // stand-in symbol, not a device address.  The device address is looked up
-// once per device with cudaGetSymbolAddress on the first call made with that
-// device current, so that first call should come before any stream capture.
-// All calls share the one array: calls that overlap on the GPU (different
-// streams, no ordering between them) race on it.  Nothing in it needs to
-// start at zero: each call writes every logit it later reads.
+// with cudaGetSymbolAddress on the first call made with a device current, and
+// again whenever the context current on that device has changed since (the
+// array is reloaded at a new address in a new context, e.g. after
+// cudaDeviceReset), so that a first call should come before any stream
+// capture.  All calls share the one array: calls that overlap on the GPU
+// (different streams, no ordering between them) race on it.  Nothing in it
+// needs to start at zero: each call writes every logit it later reads.
 namespace {
 
 constexpr size_t kNoAllocLogitsMax = 262144;
 __device__ __align__(256) float g_noalloc_logits[kNoAllocLogitsMax];
 
 constexpr int kNoAllocMaxDevices = 64;
+struct NoAllocSlot {
+  uintptr_t ctx;  // context the address was looked up in
+  float* ptr;
+};
 std::mutex g_noalloc_mu;
-float* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+NoAllocSlot g_noalloc[kNoAllocMaxDevices] = {};
 
 }  // namespace
 
@@ -239,12 +245,15 @@ extern "C" moe_status moe_route_topk_noalloc(const moe_layer_desc* desc, const v
   float* logits = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    NoAllocSlot& slot = g_noalloc[dev];
+    const uintptr_t ctx = moe::current_ctx();  // 0 before the runtime made a context on this thread
+    if (!slot.ptr || ctx == 0 || slot.ctx != ctx) {
       void* p = nullptr;
       if (cudaGetSymbolAddress(&p, g_noalloc_logits) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
-      g_noalloc_ptr[dev] = static_cast<float*>(p);
+      slot.ptr = static_cast<float*>(p);
+      slot.ctx = moe::current_ctx();
     }
-    logits = g_noalloc_ptr[dev];
+    logits = slot.ptr;
   }
   return moe::launch_route_topk(*desc, x, w_router, logit_bias, logits, topk_idx, topk_w,
                                 static_cast<cudaStream_t>(stream)) == cudaSuccess

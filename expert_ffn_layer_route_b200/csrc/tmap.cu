@@ -1,4 +1,5 @@
-// Host-side TMA tensor-map encoding through the driver entry point.
+// Host-side driver calls through the runtime's driver entry points: TMA
+// tensor-map encoding and the current context's handle.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -18,6 +19,21 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   });
   return fn;
+}
+
+uintptr_t current_ctx() {
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  });
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return 0;
+  return reinterpret_cast<uintptr_t>(c);
 }
 
 bool encode_tmap_u8(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,

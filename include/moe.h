@@ -144,16 +144,21 @@ typedef struct {
 #define MOE_ROUTER_SUM_DEPTH(d) (8 * (((d) + 2047) / 2048) + 12)
 
 /* Scratch bytes moe_layer_forward needs for `desc` (also enough for
- * moe_route_topk and moe_grouped_ffn). */
+ * moe_route_topk and moe_grouped_ffn).  No counterpart in the pages: the
+ * caller-owned scratch of this library's calls. */
 moe_status moe_workspace_size(const moe_layer_desc* desc, size_t* bytes);
 moe_status moe_workspace_layout_of(const moe_layer_desc* desc, moe_workspace_layout* out);
 
-/* Router and top-k.  logits[t][e] = sum_i x[t][i]*Wr[e][i] (+ logit_bias[e]),
+/* Router and top-k ("Mixture of experts VRAM: total vs active parameters",
+ * section "How current MoE models route each token": a dense router picks k
+ * experts per token).  logits[t][e] = sum_i x[t][i]*Wr[e][i] (+ logit_bias[e]),
  * fp32 accumulation; per token the k largest logits in descending order, the
  * lower expert index winning ties; topk_w = softmax over the selected logits
  * (equal to the softmax over all E renormalised over the selection).
  * x: bf16 [T][d]; w_router: bf16 or fp32 [E][d]; logit_bias: fp32 [E] or NULL.
- * Outputs topk_idx int32 [T][k], topk_w fp32 [T][k].  Needs `workspace`. */
+ * Outputs topk_idx int32 [T][k], topk_w fp32 [T][k].  Needs `workspace` for
+ * the fp32 logits (T*E*4 bytes; moe_route_topk_noalloc keeps them in the
+ * library instead). */
 moe_status moe_route_topk(const moe_layer_desc* desc, const void* x, const void* w_router,
                           const float* logit_bias, int32_t* topk_idx, float* topk_w,
                           void* workspace, size_t ws_bytes, void* stream);
@@ -167,21 +172,29 @@ moe_status moe_route_topk(const moe_layer_desc* desc, const void* x, const void*
  * <= 262144 (1 MiB, held on every GPU that loads the library until exit);
  * larger calls return MOE_ERR_WORKSPACE before enqueueing anything.  The
  * first call on a device looks up the array's device address (make it before
- * any stream capture).  Calls share the array: calls that overlap on the GPU
- * race.  Nothing is allocated. */
+ * any stream capture); a call that finds another context current on that
+ * device (after cudaDeviceReset, say) looks it up again.  Calls share the
+ * array: calls that overlap on the GPU race.  Nothing is allocated. */
 moe_status moe_route_topk_noalloc(const moe_layer_desc* desc, const void* x, const void* w_router,
                                   const float* logit_bias, int32_t* topk_idx, float* topk_w, void* stream);
 
-/* Stable counting sort of the T*k (token, slot) pairs by expert.
+/* Stable counting sort of the T*k (token, slot) pairs by expert (Galactus
+ * page, section "Prompt processing is a different phase": the tokens that
+ * select one expert are grouped so one weight read serves them all).
  * offsets int32 [E+1] (exclusive prefix sum of per-expert counts),
  * row_token int32 [T*k] (token of each grouped row; rows of one expert are in
- * ascending token order), inv int32 [T*k] (row of pair t*k+j).  An index
- * outside [0, E) sets MOE_ERR_DEVICE_INDEX in the device status word and the
- * pair is dropped. */
-moe_status moe_permute(const moe_layer_desc* desc, const int32_t* topk_idx, int32_t* offsets,
-                       int32_t* row_token, int32_t* inv, void* stream);
+ * ascending token order), inv int32 [T*k] (row of pair t*k+j).  With x
+ * (bf16 [T][d]) non-NULL the activation rows are also gathered into expert
+ * order: x_perm bf16 [T*k][d], x_perm[r] = x[row_token[r]] (x NULL: no
+ * gather, x_perm ignored; moe_grouped_ffn gathers by itself from x).  An
+ * index outside [0, E) sets MOE_ERR_DEVICE_INDEX in the device status word
+ * and the pair is dropped (its gathered row, if any, is zero). */
+moe_status moe_permute(const moe_layer_desc* desc, const int32_t* topk_idx, const void* x, int32_t* offsets,
+                       int32_t* row_token, int32_t* inv, void* x_perm, void* stream);
 
-/* Grouped SwiGLU expert FFN.  For every routed row r of expert e (rows
+/* Grouped SwiGLU expert FFN (gate, up and down projections: FloE verdict
+ * page, JSON field referee_report.summary; grouping: Galactus page, section
+ * "Prompt processing is a different phase").  For every routed row r of expert e (rows
  * [offsets[e], offsets[e+1])) with token t = row_token[r]:
  *   y_perm[r] = W2_e (silu(W_gate,e x_t) * (W_up,e x_t)),
  * and for every shared expert s and token t: y_shared[s][t] likewise.
@@ -193,13 +206,17 @@ moe_status moe_grouped_ffn(const moe_layer_desc* desc, const moe_weights* routed
                            const int32_t* row_token, const void* x, void* y_perm, void* y_shared,
                            void* workspace, size_t ws_bytes, void* stream);
 
-/* Weighted combine: out[t] = sum_{j<k} topk_w[t][j] * y_perm[inv[t*k+j]]
+/* Weighted combine ("Mixture of experts VRAM", section "How current MoE
+ * models route each token": routed experts weighted by the router, the shared
+ * expert on every token):
+ * out[t] = sum_{j<k} topk_w[t][j] * y_perm[inv[t*k+j]]
  *                            + sum_s y_shared[s][t]   (fp32 sum in that order),
  * out bf16 [T][d]. */
 moe_status moe_combine(const moe_layer_desc* desc, const void* y_perm, const int32_t* inv,
                        const float* topk_w, const void* y_shared, void* out, void* stream);
 
-/* The whole layer: route_topk -> permute -> grouped_ffn -> combine, all on
+/* The whole layer (the four calls above, in the pages' order):
+ * route_topk -> permute -> grouped_ffn -> combine, all on
  * `stream`, scratch in `workspace` (layout: moe_workspace_layout_of). */
 moe_status moe_layer_forward(const moe_layer_desc* desc, const void* x, const void* w_router,
                              const float* logit_bias, const moe_weights* routed,
@@ -238,14 +255,22 @@ typedef struct {
   double copy_ms; /* sum of completed copy durations (events) */
 } moe_cache_stats_t;
 
+/* Allocates the HBM slots (slots_per_layer per layer), the pinned bank
+ * (unless given), the copy stream and events ("Running MoE LLMs on a single
+ * GPU: what expert offloading actually costs", section "Inside expert
+ * paging": stable logical slots, physical residency below them). */
 moe_status moe_cache_init(moe_cache** cache, const moe_cache_desc* desc);
 /* Host pointer to layer `layer`, expert `e` in the bank (to fill it). */
 void* moe_cache_host_expert(moe_cache* cache, int32_t layer, int32_t e);
 /* Device base of the slot pool of `layer` (slot s at base + s*expert_bytes). */
 void* moe_cache_slot_base(moe_cache* cache, int32_t layer);
+/* Start copies of the listed experts of `layer` (host list) on the copy
+ * stream (FloE verdict page, referee_report.summary: prefetch from the
+ * current hidden state with asynchronous transfer). */
 moe_status moe_cache_prefetch(moe_cache* cache, int32_t layer, const int32_t* experts /*host*/,
                               int32_t n);
-/* Make `experts` (host list) of `layer` resident, write the layer's logical ->
+/* (Expert paging, same page and section; LRU: related-papers feed.)
+ * Make `experts` (host list) of `layer` resident, write the layer's logical ->
  * slot map (int32 [n_experts], -1 = absent) to slot_map_dev on `compute`
  * stream, and make `compute` wait for the copies it needs.  At most
  * slots_per_layer experts are resident at once: with a longer list the map
@@ -257,7 +282,12 @@ moe_status moe_cache_lookup(moe_cache* cache, int32_t layer, const int32_t* expe
 moe_status moe_cache_release(moe_cache* cache, int32_t layer, void* compute_stream);
 /* Host copy of the current slot map of `layer` (int32 [n_experts]). */
 moe_status moe_cache_slot_map(const moe_cache* cache, int32_t layer, int32_t* out /*host*/);
+/* Counters since init: lookups, hits, misses, evictions, prefetches issued
+ * and used, bytes copied, summed copy time (the hit rate and H2D rate the
+ * offloading pages report; "Running MoE LLMs on a single GPU", section "Inside
+ * expert paging"). */
 moe_status moe_cache_stats(moe_cache* cache, moe_cache_stats_t* out);
+/* Waits for the cache's copies, frees what moe_cache_init allocated. */
 moe_status moe_cache_destroy(moe_cache* cache);
 
 /* ------------------------------------------------------------------------

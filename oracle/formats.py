@@ -39,8 +39,25 @@ def _as_np(a) -> np.ndarray:
 
 
 def bf16_bits_to_f64(bits) -> np.ndarray:
-    """bf16 raw 16-bit patterns -> float64, from the field definition."""
-    b = _as_np(bits).astype(np.int64) & 0xFFFF
+    """bf16 raw 16-bit patterns -> float64, from the field definition (through
+    the definition's table of all 65536 patterns: same values, one lookup per
+    element)."""
+    b = _as_np(bits).astype(np.uint16)
+    return _bf16_table()[b]
+
+
+_BF16_TABLE = None
+
+
+def _bf16_table() -> np.ndarray:
+    global _BF16_TABLE
+    if _BF16_TABLE is None:
+        _BF16_TABLE = _bf16_fields_to_f64(np.arange(65536, dtype=np.int64))
+    return _BF16_TABLE
+
+
+def _bf16_fields_to_f64(b: np.ndarray) -> np.ndarray:
+    """sign, 8-bit exponent (bias 127, 0 = subnormal, 255 = inf/NaN), 7-bit mantissa."""
     s = (b >> 15) & 1
     e = (b >> 7) & 0xFF
     m = b & 0x7F

@@ -92,14 +92,29 @@ def run_steps(dlay, stream=None):
     return {"out": out, "idx": idx, "gates": gw, "offsets": offs, "row_token": rtok, "inv": inv, "y": y}
 
 
-def check_routing(hlay, idx_gpu, gates_gpu, tokens=None):
+def _routing_only(hlay, tokens, chain):
+    """The oracle's routing of the given tokens (no expert FFN)."""
+    shape = hlay["shape"]
+    x = OL.to_f64(hlay["x"])
+    tok = np.arange(x.shape[0]) if tokens is None else np.asarray(list(tokens), dtype=np.int64)
+    x = x[tok]
+    wr = OL.to_f64(hlay["router"])
+    b = OL.to_f64(hlay["bias"]) if hlay.get("bias") is not None else None
+    logits = OL.router_logits(x, wr, b)
+    idx, gates, margin = OL.topk_select(logits, shape.top_k)
+    beta = OL.logit_error_bound(x, wr, b, chain)
+    return {"idx": idx, "gates": gates, "logits": logits, "margin": margin, "beta": beta, "tokens": tok}
+
+
+def check_routing(hlay, idx_gpu, gates_gpu, tokens=None, values=True):
     """Bit-exact indices for unique tokens, validity for the others.
 
     Returns (ref, n_ambiguous) where ref is the oracle run (forced to the
-    GPU's choice where the choice is not unique)."""
+    GPU's choice where the choice is not unique).  values=False checks the
+    routing alone (no expert FFN in the oracle)."""
     shape = hlay["shape"]
     chain = moe.router_sum_depth(shape.d_model)
-    ref = OL.moe_layer(hlay, tokens=tokens, chain=chain)
+    ref = OL.moe_layer(hlay, tokens=tokens, chain=chain) if values else _routing_only(hlay, tokens, chain)
     idx_g = idx_gpu.cpu().numpy()
     if tokens is not None:
         idx_g = idx_g[np.asarray(list(tokens))]
@@ -116,7 +131,10 @@ def check_routing(hlay, idx_gpu, gates_gpu, tokens=None):
             assert np.all(np.diff(lg[p, ch]) <= 2 * beta[p])
         forced = np.zeros((hlay["x"].shape[0], shape.top_k), dtype=np.int32)
         forced[ref["tokens"]] = idx_g
-        ref = OL.moe_layer(hlay, forced_idx=forced, tokens=tokens, chain=chain)
+        if values:
+            ref = OL.moe_layer(hlay, forced_idx=forced, tokens=tokens, chain=chain)
+        else:
+            ref = dict(ref, idx=idx_g, gates=OL.gates_for(ref["logits"], idx_g))
     g = gates_gpu.cpu().double().numpy()
     if tokens is not None:
         g = g[np.asarray(list(tokens))]

@@ -153,11 +153,44 @@ def test_out_of_range_expert_index_sets_status():
     offs = torch.empty(shape.n_experts + 1, dtype=torch.int32, device="cuda")
     rtok = torch.empty(8, dtype=torch.int32, device="cuda")
     inv = torch.empty(8, dtype=torch.int32, device="cuda")
-    moe.moe_permute(desc, idx, offs, rtok, inv)
+    x = mi.draw_tokens(4, shape.d_model, 3, "cuda")
+    xp = torch.full((8, shape.d_model), 7.0, dtype=torch.bfloat16, device="cuda")
+    moe.moe_permute(desc, idx, offs, rtok, inv, x=x, x_perm=xp)
     assert moe.moe_get_last_error() == 9
     assert inv.cpu().tolist()[3] == -1
     assert offs.cpu().tolist()[-1] == 7
     assert moe.moe_get_last_error() == 0  # cleared
+    # the seven grouped rows are gathered; the dropped pair's row has no source and is zero
+    assert torch.equal(xp[:7], x[rtok[:7].long()])
+
+
+@pytest.mark.parametrize("shape,T", [(mi.GPTOSS.replace(n_experts=16), 13), (mi.KIMI, 40), (mi.TINY, 0)],
+                         ids=["mxfp4_E16_T13", "kimi_T40", "empty"])
+def test_permute_gathers_rows_in_expert_order(shape, T):
+    """moe_permute with x: offsets / row_token / inv bit-exact against the
+    oracle's stable counting sort, and x_perm[r] = x[row_token[r]] bit for bit."""
+    import expert_ffn_layer_route_b200 as moe
+    from oracle import layer as OL
+    desc = moe.make_desc(shape, T)
+    k, E = shape.top_k, shape.n_experts
+    gen = torch.Generator().manual_seed(T + 5)
+    idx = torch.stack([torch.randperm(E, generator=gen)[:k] for _ in range(T)]).to(torch.int32) if T else \
+        torch.zeros(0, k, dtype=torch.int32)
+    x = mi.draw_tokens(T, shape.d_model, 9, "cuda")
+    offs = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    rtok = torch.empty(max(T * k, 1), dtype=torch.int32, device="cuda")
+    inv = torch.empty(max(T * k, 1), dtype=torch.int32, device="cuda")
+    xp = torch.empty(max(T * k, 1), shape.d_model, dtype=torch.bfloat16, device="cuda")
+    moe.moe_permute(desc, idx.cuda(), offs, rtok, inv, x=x, x_perm=xp)
+    torch.cuda.synchronize()
+    assert moe.moe_get_last_error() == 0
+    c, o, rt, iv = OL.permute(idx.numpy(), E)
+    assert np.array_equal(offs.cpu().numpy(), o)
+    if T == 0:
+        return
+    assert np.array_equal(rtok.cpu().numpy(), rt)
+    assert np.array_equal(inv.cpu().numpy(), iv)
+    assert torch.equal(xp.cpu(), x.cpu()[torch.from_numpy(rt).long()])
 
 
 # ------------------------------------------------------------ full sizes ----
@@ -200,17 +233,36 @@ def test_full_size_routing_exact(shape, T):
     assert np.all(np.abs(g[uniq] - rg[uniq]) <= 1e-5 + 2 * rg[uniq] * beta[uniq, None])
 
 
-@pytest.mark.parametrize("shape,T,tokens", [(mi.GPTOSS, 64, [0, 13, 37, 63]), (mi.GPTOSS, 1, [0]),
-                                            (mi.KIMI, 128, [5, 77, 127]), (mi.BANK, 16, [0, 9, 15])])
-def test_full_size_layer_sampled_tokens(shape, T, tokens):
-    """Whole layer at the measured size (launch configuration of the benchmark);
-    the oracle recomputes a sample of tokens."""
+FULL_VALUE_CASES = [
+    # shape, T, tokens compared (None: every token; n: a seeded subset of n)
+    (mi.GPTOSS, 1, None), (mi.GPTOSS, 8, None), (mi.GPTOSS, 32, None), (mi.GPTOSS, 64, None),
+    (mi.KIMI, 1, None), (mi.KIMI, 8, None), (mi.KIMI, 32, None), (mi.KIMI, 128, 64),
+    (mi.BANK, 16, None),
+]
+
+
+def _token_subset(T, n, seed):
+    if n is None or n >= T:
+        return None
+    return sorted(np.random.default_rng(seed).choice(T, n, replace=False).tolist())
+
+
+@pytest.mark.parametrize("shape,T,n_tok", FULL_VALUE_CASES,
+                         ids=[f"{c[0].name}_T{c[1]}" for c in FULL_VALUE_CASES])
+def test_full_size_layer_values(shape, T, n_tok):
+    """Whole layer at the measured sizes, in the launch configurations the
+    benchmark times (column groups per pass, blocks per SM, half-height items
+    and dynamic item claiming all follow T): routing bit-exact on every token,
+    outputs against the oracle on every token (a seeded subset of 64 at
+    Kimi T=128)."""
     hl, dl = _layer(shape, T, 12, device="cuda")
     res = H.run_layer(dl)
+    tokens = _token_subset(T, n_tok, T)
     ref, n_amb = H.check_routing(hl, res["idx"], res["gates"], tokens=tokens)
     H.check_permutation(res, shape)
     rel = H.check_output(res["out"], ref["out"], tokens=tokens)
-    print(f"{shape.name} T={T}: rel err {rel:.2e} on {len(tokens)} tokens, ambiguous {n_amb}")
+    n = T if tokens is None else len(tokens)
+    print(f"{shape.name} T={T}: rel err {rel:.2e} on {n} tokens, ambiguous {n_amb}")
 
 
 # --------------------------------------------------- tensor-core GEMM path ----
@@ -239,14 +291,28 @@ def test_gemm_path_matches_oracle_and_stream_path(name, shape, T, monkeypatch):
 
 
 def test_gemm_path_full_size_prefill_sampled():
-    """Mixtral-shaped prefill (T=4096) through the default path (tensor-core GEMM)."""
+    """Mixtral-shaped prefill (T=4096) through the default path (tensor-core
+    GEMM): routing and permutation bit-exact on every token, outputs against
+    the oracle on a seeded subset of 512 tokens (which touches every m-tile of
+    every expert)."""
     hl, dl = _layer(mi.MIXTRAL, 4096, 12, device="cuda")
     res = H.run_layer(dl)
-    tokens = [0, 1001, 2047, 4095]
-    ref, n_amb = H.check_routing(hl, res["idx"], res["gates"], tokens=tokens)
+    ref_all, n_amb_all = H.check_routing(hl, res["idx"], res["gates"], tokens=None, values=False)
     H.check_permutation(res, mi.MIXTRAL)
+    tokens = _token_subset(4096, 512, 4096)
+    ref, n_amb = H.check_routing(hl, res["idx"], res["gates"], tokens=tokens)
     rel = H.check_output(res["out"], ref["out"], tokens=tokens)
-    print(f"mixtral T=4096: rel err {rel:.2e} on {len(tokens)} tokens, ambiguous {n_amb}")
+    # the subset reaches every 128-row m-tile of every expert
+    row_of = res["inv"].cpu().numpy().reshape(4096, 2)
+    offs = res["offsets"].cpu().numpy()
+    hit = set()
+    for t in tokens:
+        for r in row_of[t]:
+            e = int(np.searchsorted(offs, r, side="right") - 1)
+            hit.add((e, (int(r) - int(offs[e])) // 128))
+    tiles = {(e, m) for e in range(8) for m in range((int(offs[e + 1] - offs[e]) + 127) // 128)}
+    assert hit == tiles
+    print(f"mixtral T=4096: rel err {rel:.2e} on {len(tokens)} tokens, ambiguous {n_amb_all} of 4096")
 
 
 def test_bounded_wait_times_out_with_status_and_context_survives():

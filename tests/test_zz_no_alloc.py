@@ -50,6 +50,29 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
     assert moe.moe_get_last_error() == 0
 
 
+def test_noalloc_at_its_size_limit_matches_both_references():
+    """The largest call the scratch holds (T * n_experts = 261888 of 262144
+    logits) twice in a row: indices bit-exact and gates within GATE_TOL of the
+    workspace entry point, and the expert choice against the fp64 oracle."""
+    from oracle import layer as OL
+    shape = mi.KIMI
+    T = 262144 // shape.n_experts
+    for rep in range(2):
+        i_ref, g_ref, i_na, g_na = _both(shape, T, 25)
+        assert torch.equal(i_na, i_ref)
+        assert torch.allclose(g_na, g_ref, rtol=0, atol=GATE_TOL)
+    x, router, bias = _inputs(shape, T, 25)
+    xs, wr, b = OL.to_f64(x.cpu()), OL.to_f64(router.cpu()), OL.to_f64(bias.cpu())
+    logits = OL.router_logits(xs, wr, b)
+    ridx, rg, margin = OL.topk_select(logits, shape.top_k)
+    beta = OL.logit_error_bound(xs, wr, b, moe.router_sum_depth(shape.d_model))
+    uniq = margin > 2 * beta
+    assert np.array_equal(i_na.cpu().numpy()[uniq], ridx[uniq])
+    g = g_na.cpu().double().numpy()
+    assert np.all(np.abs(g[uniq] - rg[uniq]) <= GATE_TOL + 2 * rg[uniq] * beta[uniq, None])
+    assert moe.moe_get_last_error() == 0
+
+
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     shape = mi.KIMI  # 384 experts
     T = 262144 // shape.n_experts + 1
