@@ -37,7 +37,7 @@ METRIC = "MoE-layer tokens/s and achieved HBM GB/s (decode) / TFLOPS (prefill) v
 SHAPE = mi.GPTOSS
 PROFILE_EVERY = 10
 DEFAULT_TOKENS = {"tiny": 16, "gptoss_decode": 64, "mixtral_prefill": 4096, "kimi_decode": 128,
-                  "offload_bank": 16}
+                  "offload_bank": 16, "mixtral_prefill_mxfp4": 4096}
 L2_BYTES = 126 * 2 ** 20
 
 
@@ -357,8 +357,6 @@ def run_ours(args):
     layer_bytes = (distinct + S) * (b13 + b2) + router_bytes + act_bytes
     rows = T * k + S * T
     layer_flops = 2.0 * rows * 3 * d * f + 2.0 * T * d * shape.n_experts
-    tensor_path = shape.wdtype == "bf16" and T * k >= 64 * shape.n_experts
-    kname = "ffn_gemm_stage1_gate_up" if tensor_path else "ffn_stage1_gate_up"
     stage1_bytes = (distinct + S) * b13 + rows * d * 2 + rows * f * 2
     stage1_flops = 2.0 * rows * d * 2 * f
 
@@ -423,6 +421,11 @@ def run_ours(args):
 
     if rank == 0:
         pk = peaks()
+        # the stage-1 kernel that ran: the tensor-core GEMM (bf16 or 4-bit
+        # weights) for prefill-sized groups, else the weight-streaming kernel
+        kname = next((kk for kk in ("ffn_gemm_stage1_gate_up", "ffn_gemm_q4_stage1_gate_up") if kk in prof),
+                     "ffn_stage1_gate_up")
+        tensor_path = kname != "ffn_stage1_gate_up"
         s1 = prof.get(kname, (0, 0.0))
         s1_ms = s1[1] / max(s1[0], 1)
         step_s = ms / args.steps * 1e-3
@@ -473,10 +476,13 @@ def run_ours(args):
 
 
 def run_offload(args):
-    """Offloaded bank: decode steps through --bank-layers NVFP4 layers whose experts
-    live in pinned host memory, 25% of each layer resident in HBM under LRU, with
-    next-layer prefetch.  Reports hit rate, H2D GB/s against a measured pinned
-    host-to-device copy peak, and tokens/s of the layer stack."""
+    """Offloaded bank: decode steps through --bank-layers NVFP4 layers (default
+    all 48) whose experts live in pinned host memory, 25% of each layer
+    resident in HBM under LRU, with next-layer prefetch.  Reports hit rate,
+    H2D GB/s against a measured pinned host-to-device copy peak, tokens/s of
+    the layer stack, and the copy time prefetch hides: a second run of
+    --bank-noprefetch-steps steps without prefetch, and the time of one layer
+    with every expert resident (compute alone)."""
     import torch
     import expert_ffn_layer_route_b200 as moe
     from expert_ffn_layer_route_b200.offload import OffloadedBank
@@ -499,24 +505,54 @@ def run_offload(args):
     del hb, db
     bank = OffloadedBank(shape, L, mi.BANK_SLOTS_PER_LAYER, T)
     t0 = time.perf_counter()
+    resident_ms = None
     for l in range(L):
-        bank.fill_layer(l, mi.bank_layer(shape, l, 0, dev))
+        lay = mi.bank_layer(shape, l, 0, dev)
+        bank.fill_layer(l, lay)
+        if l == 0:
+            # one layer with all 256 experts resident in HBM: the compute alone
+            desc = moe.make_desc(shape, T)
+            ws = torch.empty(moe.moe_workspace_size(desc), dtype=torch.uint8, device=dev)
+            out = torch.empty(T, shape.d_model, dtype=torch.bfloat16, device=dev)
+            w = moe.make_weights(lay["experts"])
+            xs = [mi.bank_step_tokens(10_000 + i, T, shape.d_model, 0, dev) for i in range(8)]
+            for i in range(5):
+                moe.moe_layer_forward(desc, xs[i % 8], lay["router"], lay["bias"], w, None, out, ws)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for i in range(40):
+                moe.moe_layer_forward(desc, xs[i % 8], lay["router"], lay["bias"], w, None, out, ws)
+            b.record()
+            torch.cuda.synchronize()
+            resident_ms = a.elapsed_time(b) / 40
+            del ws, out, w
+        del lay
     fill_s = time.perf_counter() - t0
     for s_ in range(args.warmup):
         bank.decode_step(mi.bank_step_tokens(s_, T, shape.d_model, 0, dev))
     torch.cuda.synchronize()
-    st0 = bank.stats()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    xs = [mi.bank_step_tokens(args.warmup + s_, T, shape.d_model, 0, dev) for s_ in range(args.steps)]
-    e0.record()
-    for s_ in range(args.steps):
-        bank.decode_step(xs[s_])
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    st1 = bank.stats()
-    d = {k: st1[k] - st0[k] for k in st1}
+
+    def timed(n, first, prefetch):
+        st0 = bank.stats()
+        xs = [mi.bank_step_tokens(first + s_, T, shape.d_model, 0, dev) for s_ in range(n)]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for s_ in range(n):
+            bank.decode_step(xs[s_], prefetch=prefetch)
+        e1.record()
+        torch.cuda.synchronize()
+        st1 = bank.stats()
+        return e0.elapsed_time(e1), {k: st1[k] - st0[k] for k in st1}
+
+    clocks = ClockSampler()
+    clocks.start()
+    time.sleep(0.3)
+    ms, d = timed(args.steps, args.warmup, True)
+    n_np = args.bank_noprefetch_steps
+    ms_np, d_np = timed(n_np, args.warmup + args.steps, False) if n_np > 0 else (None, None)
+    clk = clocks.stop()
     h2d = d["bytes_h2d"] / (ms * 1e-3) / 1e9
+    per_layer = ms / args.steps / L
     line = {
         "metric": METRIC, "value": T * args.steps / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
@@ -532,10 +568,98 @@ def run_offload(args):
                     "misses": d["misses"], "prefetch_issued": d["prefetch_issued"],
                     "prefetch_used": d["prefetch_used"], "bytes_h2d_per_step": d["bytes_h2d"] / args.steps,
                     "copy_ms_per_step": d["copy_ms"] / args.steps, "h2d_gbs": h2d,
-                    "ms_per_layer": ms / args.steps / L},
+                    "ms_per_layer": per_layer, "resident_ms_per_layer": resident_ms,
+                    "exposed_ms_per_layer": per_layer - resident_ms if resident_ms is not None else None},
+        "clocks": clk,
     }
+    if ms_np is not None:
+        pl_np = ms_np / n_np / L
+        line["offload_without_prefetch"] = {
+            "steps": n_np, "ms_per_layer": pl_np, "hit_rate": d_np["hits"] / max(d_np["lookups"], 1),
+            "bytes_h2d_per_step": d_np["bytes_h2d"] / n_np,
+            "exposed_ms_per_layer": pl_np - resident_ms if resident_ms is not None else None,
+            "tokens_per_s": T * n_np / (ms_np * 1e-3)}
     print(json.dumps(line), flush=True)
     bank.close()
+    return 0
+
+
+def run_verify(args):
+    """Speculative verification blocks on the gpt-oss-shaped decode layer:
+    n_seq sequences each verify depth drafted tokens plus their own position
+    in one layer call (T = n_seq * (depth + 1) positions that read the union of
+    their experts once), against ordinary decode of the same sequences (T =
+    n_seq, one position each).  Accepted output per block follows seeded
+    accept flags (probability alpha per draft, stopping at the first
+    rejection).  Reports accepted tokens/s and layer bytes per accepted token
+    for both."""
+    import torch
+    import expert_ffn_layer_route_b200 as moe
+    from expert_ffn_layer_route_b200 import verify as V
+    shape = mi.GPTOSS
+    nseq, depth, rho, alpha = args.verify_seqs, args.verify_depth, args.verify_rho, args.verify_alpha
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    lay = mi.draw_layer(shape, 1, seed=1000, device=dev)
+    routed = moe.make_weights(lay["experts"])
+    b13, b2 = expert_bytes_split(shape)
+    stream = torch.cuda.current_stream(dev)
+
+    def measure(T, xs):
+        desc = moe.make_desc(shape, T)
+        ws = torch.empty(moe.moe_workspace_size(desc), dtype=torch.uint8, device=dev)
+        out = torch.empty(T, shape.d_model, dtype=torch.bfloat16, device=dev)
+        for i in range(args.warmup):
+            moe.moe_layer_forward(desc, xs[i % len(xs)], lay["router"], None, routed, None, out, ws, stream)
+        torch.cuda.synchronize()
+        L = moe.moe_workspace_layout_of(desc)
+        distinct = []
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            moe.moe_layer_forward(desc, xs[i % len(xs)], lay["router"], None, routed, None, out, ws, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        for x in xs:  # experts each input reads (union over its positions), untimed
+            moe.moe_layer_forward(desc, x, lay["router"], None, routed, None, out, ws, stream)
+            offs = ws[L.offsets: L.offsets + 4 * (shape.n_experts + 1)].view(torch.int32).cpu().numpy()
+            distinct.append(int((np.diff(offs) > 0).sum()))
+        d_mean = float(np.mean(distinct))
+        layer_bytes = d_mean * (b13 + b2) + shape.n_experts * shape.d_model * 2 + 2 * T * shape.d_model * 2
+        return ms, d_mean, layer_bytes
+
+    n_inputs = 8
+    xv = [mi.draw_verify_tokens(nseq, depth, shape.d_model, rho, 2000 + i, dev) for i in range(n_inputs)]
+    x1 = [xi.view(nseq, depth + 1, -1)[:, 0].contiguous() for xi in xv]  # the sequences' own positions
+    clocks = ClockSampler()
+    clocks.start()
+    time.sleep(0.3)
+    ms_v, dv, bytes_v = measure(nseq * (depth + 1), xv)
+    ms_o, do, bytes_o = measure(nseq, x1)
+    clk = clocks.stop()
+    acc = [sum(V.accepted_tokens(a) for a in mi.draw_accepts(nseq, depth, alpha, 3000 + i).tolist())
+           for i in range(args.steps)]
+    acc_mean = float(np.mean(acc))
+    value = acc_mean / (ms_v * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_v, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"verify: gpt-oss-shaped decode layer (d_model=2880 E=128 top-4 d_ff=2880 MXFP4), "
+                               f"{nseq} sequences x (1 + {depth} drafted) positions per call, positions of a "
+                               f"sequence correlated (rho={rho}), accept probability {alpha} per draft",
+                   "tokens": nseq * (depth + 1), "l2": "inputs larger than L2 (each call reads >= 1 GB of experts)"},
+        "verify": {"accepted_per_step": acc_mean, "expected_accepted_per_step": nseq * V.expected_accepted_tokens(depth, alpha),
+                   "distinct_experts": dv, "layer_bytes": bytes_v,
+                   "bytes_per_accepted_token": V.bytes_per_accepted_token(bytes_v, acc_mean),
+                   "ms_per_call": ms_v},
+        "ordinary_decode": {"tokens_per_step": nseq, "distinct_experts": do, "layer_bytes": bytes_o,
+                            "bytes_per_token": V.bytes_per_accepted_token(bytes_o, nseq), "ms_per_call": ms_o,
+                            "tokens_per_s": nseq / (ms_o * 1e-3)},
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
     return 0
 
 
@@ -545,10 +669,16 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--tokens", type=int, default=0, help="tokens per step (default: the workload's)")
-    ap.add_argument("--workload", choices=sorted(DEFAULT_TOKENS), default="gptoss_decode")
+    ap.add_argument("--workload", choices=sorted(DEFAULT_TOKENS) + ["verify"], default="gptoss_decode")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--bank-layers", type=int, default=8, help="layers of the offloaded bank (of 48)")
+    ap.add_argument("--bank-layers", type=int, default=mi.BANK_LAYERS, help="layers of the offloaded bank (of 48)")
+    ap.add_argument("--bank-noprefetch-steps", type=int, default=16,
+                    help="offload_bank: steps of a second run without prefetch (0: none)")
+    ap.add_argument("--verify-seqs", type=int, default=16, help="verify: sequences per call")
+    ap.add_argument("--verify-depth", type=int, default=3, help="verify: drafted tokens per sequence")
+    ap.add_argument("--verify-rho", type=float, default=0.5, help="verify: correlation of a sequence's positions")
+    ap.add_argument("--verify-alpha", type=float, default=0.7, help="verify: accept probability per draft")
     ap.add_argument("--no-kernel-timing", action="store_true",
                     help="no per-kernel CUDA events in the timed region (the roofline fields are then empty)")
     args = ap.parse_args()
@@ -558,6 +688,8 @@ def main():
         return run_reference(args)
     if args.workload == "offload_bank":
         return run_offload(args)
+    if args.workload == "verify":
+        return run_verify(args)
     return run_ours(args)
 
 

@@ -160,8 +160,25 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
   __half* hq = reinterpret_cast<__half*>(ws + L.hq);
   int32_t* hexp = reinterpret_cast<int32_t*>(ws + L.hexp);
-  float* gbias = f == MOE_W_INT4_G128 ? reinterpret_cast<float*>(ws + L.gbias) : nullptr;
-  const int mode = !q ? 2 : (f == MOE_W_INT4_G128 ? 1 : 0);
+  // Path: the tcgen05 grouped GEMM when experts average at least 64 rows
+  // (prefill-sized groups; bf16 weights, or 4-bit weights decoded to 16-bit
+  // tiles in shared memory), else the weight-streaming kernel.
+  // MOE_FFN_PATH=stream|gemm overrides the choice where both can run.
+  const bool gemm_ok = q ? (gemm_q4_supported(f, F, D, true) && gemm_q4_supported(f, D, F, false))
+                         : (gemm_path_supported(f, F, D, true) && gemm_path_supported(f, D, F, false));
+  bool use_gemm = gemm_ok && (int64_t)T * k >= 64LL * E;
+  if (const char* e = getenv("MOE_FFN_PATH")) {
+    if (!strcmp(e, "stream")) use_gemm = false;
+    if (!strcmp(e, "gemm")) use_gemm = gemm_ok;
+  }
+  // Activation rows: bf16 copies (bf16 weights; MXFP4 on the tensor-core
+  // path), fp16 scaled by a power of two per row (the 4-bit formats
+  // otherwise), for the streaming INT4 decode also reordered with the
+  // per-group constants.
+  const bool q_bf16_acts = q && use_gemm && gemm_q4_bf16_activations(f);
+  const bool int4_stream = f == MOE_W_INT4_G128 && !use_gemm;
+  float* gbias = int4_stream ? reinterpret_cast<float*>(ws + L.gbias) : nullptr;
+  const int mode = (!q || q_bf16_acts) ? 2 : (int4_stream ? 1 : 0);
   // activation rows in expert order (routed rows, then every token once per shared expert)
   // (also zeroes the work counters of both FFN stages)
   int32_t* ctr = reinterpret_cast<int32_t*>(ws + L.ctr);
@@ -198,15 +215,6 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
     a.K = (int)K;
     a.offsets = offsets;
   };
-  // Path: the tcgen05 grouped GEMM when experts average at least 64 rows
-  // (prefill-sized groups; bf16 weights), else the weight-streaming kernel.
-  // MOE_FFN_PATH=stream|gemm overrides the choice where both can run.
-  bool use_gemm = gemm_path_supported(f, F, D, true) && gemm_path_supported(f, D, F, false) &&
-                  (int64_t)T * k >= 64LL * E;
-  if (const char* e = getenv("MOE_FFN_PATH")) {
-    if (!strcmp(e, "stream")) use_gemm = false;
-    if (!strcmp(e, "gemm")) use_gemm = gemm_path_supported(f, F, D, true) && gemm_path_supported(f, D, F, false);
-  }
   auto to_gemm = [&](const FfnArgs& s) {
     GemmArgs g;
     std::memset(&g, 0, sizeof(g));
@@ -223,6 +231,38 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
     g.out_shared = s.out_shared;
     return g;
   };
+  // the 4-bit tensor-core stages: argument block and pointers
+  auto to_q4 = [&](const FfnArgs& s, const FfnPointers& p, bool stage1, GemmQ4Pointers& qp) {
+    GemmQ4Args g;
+    std::memset(&g, 0, sizeof(g));
+    std::memset(&qp, 0, sizeof(qp));
+    g.offsets = s.offsets;
+    g.slot_map = s.slot_map;
+    g.n_phys = s.n_phys;
+    g.n_shared = s.n_shared;
+    g.E = s.E;
+    g.T = s.T;
+    g.k = s.k;
+    g.N = s.N;
+    g.K = s.K;
+    g.gsc = s.gsc;
+    g.gsc_sh = s.gsc_sh;
+    g.xexp = q_bf16_acts ? nullptr : s.xexp;
+    g.out_routed = s.out_routed;
+    g.out_shared = s.out_shared;
+    qp.w = p.w;
+    qp.stride_w = p.stride_w;
+    qp.s = s.s;
+    qp.stride_s = s.stride_s;
+    qp.w_sh = p.w_sh;
+    qp.stride_w_sh = p.stride_w_sh;
+    qp.s_sh = s.s_sh;
+    qp.stride_s_sh = s.stride_s_sh;
+    qp.x = p.x;
+    qp.rows_total = p.rows_total;
+    (void)stage1;
+    return g;
+  };
   FfnArgs a1;
   FfnPointers p1;
   fill(a1, p1, true);
@@ -233,26 +273,33 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
   a1.out_routed = h;
   a1.out_shared = nullptr;
   int unsup = 0;
-  if (use_gemm)
+  GemmQ4Pointers qp;
+  if (use_gemm && q)
+    err = launch_ffn_gemm_q4(f, true, to_q4(a1, p1, true, qp), qp, di.sms, di.smem_optin, st, &unsup);
+  else if (use_gemm)
     err = launch_ffn_gemm(true, to_gemm(a1), p1, di.sms, di.smem_optin, st, &unsup);
   else
     err = launch_ffn_stream(f, true, a1, p1, T, di.sms, di.smem_optin, di.smem_per_sm, st, &unsup);
   if (unsup) return MOE_ERR_UNSUPPORTED;
   if (err != cudaSuccess) return MOE_ERR_CUDA;
-  if (q) {
+  // h rows for stage 2: as written (bf16) for bf16 operands, else fp16 scaled
+  const bool h_f16 = q && !q_bf16_acts;
+  if (h_f16) {
     err = launch_prep_rows(h, RT, F, mode, hq, hexp, gbias, nullptr, 0, T, nullptr, 0, st);
     if (err != cudaSuccess) return MOE_ERR_CUDA;
   }
   FfnArgs a2;
   FfnPointers p2;
   fill(a2, p2, false);
-  p2.x = q ? static_cast<const void*>(hq) : static_cast<const void*>(h);
-  a2.xexp = q ? hexp : nullptr;
+  p2.x = h_f16 ? static_cast<const void*>(hq) : static_cast<const void*>(h);
+  a2.xexp = h_f16 ? hexp : nullptr;
   a2.xbias = gbias;
   a2.work_ctr = ctr + 1;
   a2.out_routed = static_cast<__nv_bfloat16*>(y_perm);
   a2.out_shared = static_cast<__nv_bfloat16*>(y_shared);
-  if (use_gemm)
+  if (use_gemm && q)
+    err = launch_ffn_gemm_q4(f, false, to_q4(a2, p2, false, qp), qp, di.sms, di.smem_optin, st, &unsup);
+  else if (use_gemm)
     err = launch_ffn_gemm(false, to_gemm(a2), p2, di.sms, di.smem_optin, st, &unsup);
   else
     err = launch_ffn_stream(f, false, a2, p2, T, di.sms, di.smem_optin, di.smem_per_sm, st, &unsup);

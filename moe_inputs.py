@@ -71,6 +71,10 @@ MIXTRAL = LayerShape("mixtral_prefill", 4096, 8, 2, 14336, "bf16")
 KIMI = LayerShape("kimi_decode", 7168, 384, 8, 2048, "int4", n_shared=1, zipf_s=1.1)
 BANK = LayerShape("offload_bank", 4096, 256, 8, 1536, "nvfp4", zipf_s=1.1)
 
+# The Mixtral-shaped prefill layer with MXFP4 experts (4-bit prefill on the
+# tensor cores); not one of the five measured configurations above.
+MIXTRAL_MXFP4 = MIXTRAL.replace(name="mixtral_prefill_mxfp4", wdtype="mxfp4")
+
 CONFIG_TOKENS = {
     "tiny": (16,),
     "gptoss_decode": (1, 8, 32, 64),
@@ -82,7 +86,7 @@ BANK_LAYERS = 48
 BANK_SLOTS_PER_LAYER = 64  # 25% of 256 experts
 BANK_STEPS = 512
 
-CONFIGS = {c.name: c for c in (TINY, GPTOSS, MIXTRAL, KIMI, BANK)}
+CONFIGS = {c.name: c for c in (TINY, GPTOSS, MIXTRAL, KIMI, BANK, MIXTRAL_MXFP4)}
 
 
 def _gen(seed: int, device) -> torch.Generator:
@@ -262,6 +266,27 @@ def draw_layer(shape: LayerShape, T: int, seed: int = 0, device="cpu",
         lay["experts"] = draw_experts(shape, shape.n_experts, seed * 7919 + 1, device)
     lay["shared"] = draw_experts(shape, shape.n_shared, seed * 7919 + 2, device) if shape.n_shared else None
     return lay
+
+
+def draw_verify_tokens(n_seq: int, depth: int, d: int, rho: float, seed: int, device="cpu") -> torch.Tensor:
+    """Activations of ``n_seq`` speculative verification blocks of ``depth + 1``
+    positions each (the target's own position and ``depth`` drafted ones),
+    block-major: row b*(depth+1) + i is position i of sequence b.  Positions
+    of one sequence are correlated, x = sqrt(rho) u_b + sqrt(1 - rho) z_(b,i)
+    with u, z ~ N(0, 1), so that they tend to select the same experts; bf16."""
+    gen = _gen(seed ^ 0x5EC0DE, device)
+    u = torch.randn(n_seq, 1, d, generator=gen, device=device)
+    z = torch.randn(n_seq, depth + 1, d, generator=gen, device=device)
+    x = math.sqrt(rho) * u + math.sqrt(1.0 - rho) * z
+    return x.reshape(n_seq * (depth + 1), d).to(torch.bfloat16).contiguous()
+
+
+def draw_accepts(n_seq: int, depth: int, alpha: float, seed: int) -> torch.Tensor:
+    """Seeded accept flags of the drafted tokens, bool [n_seq, depth]: each
+    drafted token is accepted with probability ``alpha`` (the verifier keeps
+    the leading run of accepted drafts)."""
+    gen = _gen(seed ^ 0xACCE97, "cpu")
+    return torch.rand(n_seq, depth, generator=gen) < alpha
 
 
 def expert_bytes(shape: LayerShape) -> int:

@@ -241,6 +241,24 @@ FULL_VALUE_CASES = [
 ]
 
 
+def _tile_covering_subset(res, T, k, n, seed):
+    """n tokens: one whose row lies in each 128-row m-tile of each expert's
+    group (so that every tile the tensor-core kernel runs is checked), the rest
+    a seeded random choice."""
+    row_of = res["inv"].cpu().numpy().reshape(T, k)
+    offs = res["offsets"].cpu().numpy()
+    first = {}
+    for t in range(T):
+        for r in row_of[t]:
+            e = int(np.searchsorted(offs, r, side="right") - 1)
+            first.setdefault((e, (int(r) - int(offs[e])) // 128), t)
+    tiles = {(e, m) for e in range(len(offs) - 1) for m in range((int(offs[e + 1] - offs[e]) + 127) // 128)}
+    assert set(first) == tiles
+    chosen = set(first.values())
+    rest = [t for t in np.random.default_rng(seed).permutation(T).tolist() if t not in chosen]
+    return sorted(chosen | set(rest[: max(0, n - len(chosen))]))
+
+
 def _token_subset(T, n, seed):
     if n is None or n >= T:
         return None
@@ -263,6 +281,28 @@ def test_full_size_layer_values(shape, T, n_tok):
     rel = H.check_output(res["out"], ref["out"], tokens=tokens)
     n = T if tokens is None else len(tokens)
     print(f"{shape.name} T={T}: rel err {rel:.2e} on {n} tokens, ambiguous {n_amb}")
+
+
+@pytest.mark.parametrize("n_seq,depth", [(16, 3), (4, 2), (1, 4)])
+def test_verification_block_values_and_expert_union(n_seq, depth):
+    """A speculative verification block (n_seq sequences x (1 + depth)
+    correlated positions in one call) on the full-size gpt-oss layer: every
+    position against the oracle, and the experts the call reads (from the
+    GPU's offsets) equal to the union of the positions' oracle choices."""
+    from oracle import cost as OC
+    shape = mi.GPTOSS
+    T = n_seq * (depth + 1)
+    hl, dl = _layer(shape, T, 14, device="cuda")
+    x = mi.draw_verify_tokens(n_seq, depth, shape.d_model, 0.5, 15, "cuda")
+    hl["x"], dl["x"] = x, x
+    res = H.run_layer(dl)
+    ref, n_amb = H.check_routing(hl, res["idx"], res["gates"])
+    H.check_permutation(res, shape)
+    rel = H.check_output(res["out"], ref["out"])
+    offs = res["offsets"].cpu().numpy()
+    assert int((np.diff(offs) > 0).sum()) == OC.expert_union(ref["idx"])
+    print(f"verify n_seq={n_seq} depth={depth}: rel err {rel:.2e}, union {OC.expert_union(ref['idx'])} experts, "
+          f"ambiguous {n_amb}")
 
 
 # --------------------------------------------------- tensor-core GEMM path ----
@@ -299,20 +339,76 @@ def test_gemm_path_full_size_prefill_sampled():
     res = H.run_layer(dl)
     ref_all, n_amb_all = H.check_routing(hl, res["idx"], res["gates"], tokens=None, values=False)
     H.check_permutation(res, mi.MIXTRAL)
-    tokens = _token_subset(4096, 512, 4096)
+    tokens = _tile_covering_subset(res, 4096, 2, 512, 4096)
     ref, n_amb = H.check_routing(hl, res["idx"], res["gates"], tokens=tokens)
     rel = H.check_output(res["out"], ref["out"], tokens=tokens)
-    # the subset reaches every 128-row m-tile of every expert
-    row_of = res["inv"].cpu().numpy().reshape(4096, 2)
-    offs = res["offsets"].cpu().numpy()
-    hit = set()
-    for t in tokens:
-        for r in row_of[t]:
-            e = int(np.searchsorted(offs, r, side="right") - 1)
-            hit.add((e, (int(r) - int(offs[e])) // 128))
-    tiles = {(e, m) for e in range(8) for m in range((int(offs[e + 1] - offs[e]) + 127) // 128)}
-    assert hit == tiles
     print(f"mixtral T=4096: rel err {rel:.2e} on {len(tokens)} tokens, ambiguous {n_amb_all} of 4096")
+
+
+# ------------------------------------------ 4-bit tensor-core GEMM path ----
+
+Q4_GEMM_CASES = [
+    # 4-bit layers with prefill-sized expert groups; K multiples of 512 (MXFP4),
+    # 256 (NVFP4), 1024 (INT4); ragged groups (second 128-row half partly or
+    # not at all filled), shared expert, several weight tiles and K steps
+    ("mxfp4_gemm_ragged", mi.GPTOSS.replace(d_model=1024, d_ff=1536, n_experts=4, top_k=2), 300),
+    ("mxfp4_gemm_small_groups", mi.GPTOSS.replace(d_model=512, d_ff=512, n_experts=8, top_k=2), 290),
+    ("nvfp4_gemm", mi.BANK.replace(d_model=512, d_ff=768, n_experts=6, top_k=2), 400),
+    ("int4_gemm_shared", mi.KIMI.replace(d_model=1024, d_ff=1024, n_experts=8, top_k=2), 260),
+]
+
+
+@pytest.mark.parametrize("name,shape,T", Q4_GEMM_CASES, ids=[c[0] for c in Q4_GEMM_CASES])
+def test_q4_gemm_path_matches_oracle_and_stream_path(name, shape, T, monkeypatch):
+    """4-bit experts through the tensor-core GEMM (weights decoded once per
+    tile to 16-bit values in shared memory) against the fp64 oracle, and
+    against the streaming path on the same inputs."""
+    import expert_ffn_layer_route_b200 as moe
+    hl, dl = _layer(shape, T, 33)
+    monkeypatch.setenv("MOE_FFN_PATH", "gemm")
+    moe.moe_profile_enable(True)
+    moe.moe_profile_collect()
+    res = H.run_layer(dl)
+    prof = moe.moe_profile_collect()
+    moe.moe_profile_enable(False)
+    assert "ffn_gemm_q4_stage1_gate_up" in prof and "ffn_gemm_q4_stage2_down" in prof, sorted(prof)
+    rel, n_amb = H.full_check(hl, res)
+    monkeypatch.setenv("MOE_FFN_PATH", "stream")
+    res_s = H.run_layer(dl)
+    o1, o2 = res["out"].float(), res_s["out"].float()
+    assert (o1 - o2).abs().max().item() <= 1e-2 * o2.abs().max().item()
+    assert moe.moe_get_last_error() == 0
+    print(f"{name}: rel err {rel:.2e}, ambiguous {n_amb}")
+
+
+def test_q4_gemm_is_default_for_prefill_sized_groups():
+    """Without an override a 4-bit batch averaging >= 64 rows per expert takes
+    the tensor-core path; a decode-sized batch keeps the streaming kernel."""
+    import expert_ffn_layer_route_b200 as moe
+    shape = mi.GPTOSS.replace(d_model=512, d_ff=512, n_experts=4, top_k=2)
+    for T, want in [(256, "ffn_gemm_q4_stage1_gate_up"), (8, "ffn_stage1_gate_up")]:
+        hl, dl = _layer(shape, T, 34)
+        moe.moe_profile_enable(True)
+        moe.moe_profile_collect()
+        res = H.run_layer(dl)
+        prof = moe.moe_profile_collect()
+        moe.moe_profile_enable(False)
+        assert want in prof, (T, sorted(prof))
+        H.full_check(hl, res)
+
+
+def test_q4_gemm_full_size_mixtral_mxfp4_prefill_sampled():
+    """Mixtral-shaped prefill (T=4096) with MXFP4 experts on the tensor-core
+    path: routing bit-exact on every token, outputs against the oracle on a
+    seeded subset of 512 tokens."""
+    hl, dl = _layer(mi.MIXTRAL_MXFP4, 4096, 13, device="cuda")
+    res = H.run_layer(dl)
+    H.check_routing(hl, res["idx"], res["gates"], tokens=None, values=False)
+    H.check_permutation(res, mi.MIXTRAL_MXFP4)
+    tokens = _tile_covering_subset(res, 4096, 2, 512, 4097)
+    ref, n_amb = H.check_routing(hl, res["idx"], res["gates"], tokens=tokens)
+    rel = H.check_output(res["out"], ref["out"], tokens=tokens)
+    print(f"mixtral mxfp4 T=4096: rel err {rel:.2e} on {len(tokens)} tokens, ambiguous {n_amb}")
 
 
 def test_bounded_wait_times_out_with_status_and_context_survives():

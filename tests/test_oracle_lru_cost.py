@@ -1,8 +1,11 @@
-"""Pins for the LRU replay (a hand-worked trace) and for the decode cost
-model (the numbers printed on the Galactus page)."""
+"""Pins for the LRU replay (a hand-worked trace), for the decode cost model
+(the numbers printed on the Galactus page) and for the verification-block
+accounting (brute force over acceptance patterns, special cases)."""
+import itertools
 import json
 import os
 
+import numpy as np
 import pytest
 
 from oracle import cost
@@ -64,3 +67,53 @@ def test_cost_model_reproduces_page_numbers():
     assert t_new == w["T_new_ms"]
     assert round(cost.tokens_per_second(t_new / 1000.0), 2) == w["tok_s_new"]
     assert round(w["tok_s_new"] / w["tok_s"] - 1, 2) == w["throughput_gain_about"]
+
+
+def pin_expected_accepted(fn):
+    """The closed form against brute force over every accept/reject pattern of
+    the drafts (probability of each pattern times its output tokens), and the
+    special cases: alpha = 0 is ordinary decode (one token), alpha = 1 accepts
+    every draft."""
+    for depth in range(0, 6):
+        for alpha in (0.0, 0.3, 0.7, 0.95, 1.0):
+            brute = 0.0
+            for pat in itertools.product([0, 1], repeat=depth):
+                p = np.prod([alpha if a else 1 - alpha for a in pat]) if depth else 1.0
+                brute += p * cost.accepted_in_block(np.array(pat))
+            if abs(fn(depth, alpha) - brute) > 1e-12:
+                return False
+        if fn(depth, 0.0) != 1.0 or fn(depth, 1.0) != depth + 1:
+            return False
+    return True
+
+
+def test_expected_accepted_matches_brute_force():
+    assert pin_expected_accepted(cost.expected_accepted)
+
+
+def test_accepted_in_block_and_union():
+    assert cost.accepted_in_block(np.array([1, 1, 0, 1])) == 3  # stops at the first rejection
+    assert cost.accepted_in_block(np.array([0, 1, 1])) == 1
+    assert cost.accepted_in_block(np.array([], dtype=bool)) == 1
+    assert cost.expert_union(np.array([[3, 1], [1, 7], [3, 7]])) == 3
+    assert cost.bytes_per_accepted_token(300.0, 2.5) == 120.0
+
+
+def test_verification_pins_reject_planted_mistakes():
+    # one draft too few in the sum, and acceptance that does not stop at a rejection
+    assert not pin_expected_accepted(lambda d, a: float(sum(a ** i for i in range(d))))
+    assert not pin_expected_accepted(lambda d, a: 1.0 + d * a)
+
+
+def test_library_verification_accounting_matches_oracle():
+    """The package's verification-block counters against the oracle's pinned ones."""
+    from expert_ffn_layer_route_b200 import verify as V
+    rng = np.random.default_rng(9)
+    for _ in range(200):
+        depth = int(rng.integers(0, 7))
+        flags = rng.random(depth) < 0.6
+        assert V.accepted_tokens(flags.tolist()) == cost.accepted_in_block(flags)
+        alpha = float(rng.random())
+        assert V.expected_accepted_tokens(depth, alpha) == pytest.approx(cost.expected_accepted(depth, alpha),
+                                                                         rel=1e-14)
+    assert V.bytes_per_accepted_token(300.0, 2.5) == cost.bytes_per_accepted_token(300.0, 2.5)
