@@ -37,7 +37,8 @@ METRIC = "MoE-layer tokens/s and achieved HBM GB/s (decode) / TFLOPS (prefill) v
 SHAPE = mi.GPTOSS
 PROFILE_EVERY = 10
 DEFAULT_TOKENS = {"tiny": 16, "gptoss_decode": 64, "mixtral_prefill": 4096, "kimi_decode": 128,
-                  "offload_bank": 16, "mixtral_prefill_mxfp4": 4096}
+                  "offload_bank": 16, "mixtral_prefill_mxfp4": 4096, "mixtral_prefill_nvfp4": 4096,
+                  "mixtral_prefill_int4": 4096}
 L2_BYTES = 126 * 2 ** 20
 
 
@@ -159,6 +160,17 @@ def host_cores():
         return len(os.sched_getaffinity(0))
     except AttributeError:  # pragma: no cover
         return os.cpu_count() or 1
+
+
+def host_mem_available():
+    """MemAvailable of the host in bytes (None when unknown)."""
+    try:
+        for ln in open("/proc/meminfo"):
+            if ln.startswith("MemAvailable:"):
+                return int(ln.split()[1]) * 1024
+    except OSError:
+        pass
+    return None
 
 
 def cpu_model():
@@ -305,7 +317,8 @@ def stored_traffic(workload, T):
 def launches_per_step(prof, steps):
     """Kernel launches in the timed region: the sampled steps' launch count per
     step times the number of steps."""
-    sampled = (steps + PROFILE_EVERY - 1) // PROFILE_EVERY
+    every = PROFILE_EVERY if steps >= 10 * PROFILE_EVERY else 1
+    sampled = len([i for i in range(steps) if i > 0 and i % every == 0])
     per_step = sum(v[0] for v in prof.values()) / max(sampled, 1)
     return int(round(per_step * steps))
 
@@ -377,10 +390,13 @@ def run_ours(args):
     # per-kernel CUDA events on every PROFILE_EVERY-th step of the timed region
     # (events between launches also stop a kernel from overlapping its
     # predecessor, so they are sampled rather than put around every launch)
+    # sampled steps: every 10th of a long run, every step but the first of a
+    # short one (the first timed step is never sampled)
+    every = PROFILE_EVERY if args.steps >= 10 * PROFILE_EVERY else 1
     e0.record(stream)
     for i in range(args.steps):
         if not args.no_kernel_timing:
-            moe.moe_profile_enable(i % PROFILE_EVERY == 0)
+            moe.moe_profile_enable(i > 0 and i % every == 0)
         step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
@@ -503,6 +519,15 @@ def run_offload(args):
         torch.cuda.synchronize()
         best = max(best, (1 << 30) / (a.elapsed_time(b) * 1e-3) / 1e9)
     del hb, db
+    # the pinned bank must leave the host room: take fewer layers when it would not
+    note = None
+    per_layer_bytes = shape.n_experts * (mi.expert_bytes(shape) + 4 * 256)
+    avail = host_mem_available()
+    if avail is not None:
+        fit = int((avail - 40 * 2 ** 30) // per_layer_bytes)
+        if fit < L:
+            note = f"layers reduced from {L} to {max(fit, 1)} to fit the host's available memory ({avail / 2**30:.0f} GiB)"
+            L = max(fit, 1)
     bank = OffloadedBank(shape, L, mi.BANK_SLOTS_PER_LAYER, T)
     t0 = time.perf_counter()
     resident_ms = None
@@ -561,7 +586,7 @@ def run_offload(args):
                                f"{mi.BANK_SLOTS_PER_LAYER} HBM slots per layer (25%), LRU + next-layer prefetch, "
                                f"T={T} tokens/step, residual chain x_l+1 = x_l + out_l",
                    "tokens": T, "layers": L, "bank_bytes": L * shape.n_experts * bank.blob.size,
-                   "fill_s": round(fill_s, 1)},
+                   "fill_s": round(fill_s, 1), "host_memory_note": note},
         "roofline": {"bound": "pcie_h2d", "achieved": h2d, "peak": best, "unit": "GB/s", "frac": h2d / best,
                      "peak_source": "measured pinned cudaMemcpy, 1 GiB", "traffic": None},
         "offload": {"hit_rate": d["hits"] / max(d["lookups"], 1), "lookups": d["lookups"], "hits": d["hits"],

@@ -104,13 +104,59 @@ __host__ __device__ constexpr uint32_t idesc_f16kind(int M, int N, bool bf16) {
          ((uint32_t)(M >> 4) << 24);
 }
 
-// fp16 pair -> bf16 pair after multiplying both by f (exact when the products
-// have at most 8 significant bits and lie in bf16's range).
-__device__ __forceinline__ uint32_t f16x2_scale_to_bf16x2(uint32_t h2, float f) {
-  const __half2 h = *reinterpret_cast<const __half2*>(&h2);
-  const float2 v = __half22float2(h);
-  __nv_bfloat162 b = __floats2bfloat162_rn(v.x * f, v.y * f);
-  return *reinterpret_cast<uint32_t*>(&b);
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+// Eight E2M1 codes (nibble i = K i of the word) -> four 16-bit pairs in K
+// order (2i, 2i+1) by table lookup on the integer pipe: byte permutes pick
+// each magnitude's high (and, for bf16, low) byte from 8-entry tables, a
+// second permute interleaves them, and the code's sign bit is moved to bit
+// 15 / 31 of its pair.  Tables: E2M1 magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 as
+// bf16 (0x0000 3F00 3F80 3FC0 4000 4040 4080 40C0) or fp16 (0x0000 3800 3C00
+// 3E00 4000 4200 4400 4600, whose low bytes are all zero).  No conversion
+// instruction is used: the conversion unit's throughput would otherwise bound
+// the converters.
+template <bool kBf16>
+__device__ __forceinline__ void e2m1x8_to_16x8_lut(uint32_t w, uint32_t (&o)[4]) {
+  const uint32_t m = w & 0x77777777u;  // magnitude codes
+  const uint32_t m2 = m >> 16;
+  const uint32_t s8 = w & 0x88888888u;  // sign bits
+  const uint32_t t = s8 << 4;           // sign of the even code of byte b in the msb of byte b
+  if constexpr (kBf16) {
+    const uint32_t hA = prmt(0x3F3F3F00u, 0x40404040u, m), lA = prmt(0xC0800000u, 0xC0804000u, m);
+    const uint32_t hB = prmt(0x3F3F3F00u, 0x40404040u, m2), lB = prmt(0xC0800000u, 0xC0804000u, m2);
+    o[0] = prmt(lA, hA, 0x5140u);
+    o[1] = prmt(lA, hA, 0x7362u);
+    o[2] = prmt(lB, hB, 0x5140u);
+    o[3] = prmt(lB, hB, 0x7362u);
+  } else {
+    const uint32_t hA = prmt(0x3E3C3800u, 0x46444240u, m), hB = prmt(0x3E3C3800u, 0x46444240u, m2);
+    o[0] = prmt(hA, 0u, 0x1404u);
+    o[1] = prmt(hA, 0u, 0x3424u);
+    o[2] = prmt(hB, 0u, 0x1404u);
+    o[3] = prmt(hB, 0u, 0x3424u);
+  }
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    // byte 1 <- byte b of t (even code's sign), byte 3 <- byte b of s8 (odd code's sign)
+    const uint32_t sg = prmt(t, s8, (uint32_t)b * 0x11u | (uint32_t)(4 + b) * 0x1100u);
+    o[b] |= sg & 0x80008000u;
+  }
+}
+
+// bf16 pair (2^(e-127), 2^(e-127)) of an E8M0 scale byte (e = 0: 2^-127, a
+// bf16 subnormal; e = 255: NaN).
+__device__ __forceinline__ uint32_t e8m0_to_bf16x2(uint32_t e) {
+  const uint32_t b = e == 0u ? 0x0040u : (e == 255u ? 0x7fc0u : (e << 7));
+  return b | (b << 16);
+}
+
+__device__ __forceinline__ uint32_t hmul2_bf16_u32(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
 }
 
 // Eight INT4 codes (nibble i = K i of the word) -> four fp16 pairs in K order
@@ -462,24 +508,19 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
         for (int g = 0; g < 8; ++g) {  // granule g: K = 8g .. 8g+7 of the step
           uint32_t o[4];
           if constexpr (F == kMXFP4) {
-            // E8M0 byte of the 32-block holding this granule
-            const float f = e8m0_to_f32((sbits >> (8 * (g >> 2))) & 0xffu);  // 2^(e-127)
-            uint32_t h0, h1, h2, h3;
-            e2m1x8_to_f16x8(cw[g], h0, h1, h2, h3);
-            o[0] = f16x2_scale_to_bf16x2(h0, f);
-            o[1] = f16x2_scale_to_bf16x2(h1, f);
-            o[2] = f16x2_scale_to_bf16x2(h2, f);
-            o[3] = f16x2_scale_to_bf16x2(h3, f);
+            // E8M0 byte of the 32-block holding this granule, as a bf16 pair;
+            // E2M1 x 2^(e-127) is exact in bf16
+            const uint32_t s2 = e8m0_to_bf16x2((sbits >> (8 * (g >> 2))) & 0xffu);
+            e2m1x8_to_16x8_lut<true>(cw[g], o);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) o[q] = hmul2_bf16_u32(o[q], s2);
           } else if constexpr (F == kNVFP4) {
             // E4M3 byte of the 16-block holding this granule, as an fp16 pair
             const uint32_t e = (sbits >> (8 * (g >> 1))) & 0xffu;
             const uint32_t s2 = e4m3x2_to_f16x2(e | (e << 8));
-            uint32_t h0, h1, h2, h3;
-            e2m1x8_to_f16x8(cw[g], h0, h1, h2, h3);
-            o[0] = hmul2_u32(h0, s2);
-            o[1] = hmul2_u32(h1, s2);
-            o[2] = hmul2_u32(h2, s2);
-            o[3] = hmul2_u32(h3, s2);
+            e2m1x8_to_16x8_lut<false>(cw[g], o);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) o[q] = hmul2_u32(o[q], s2);
           } else {
             // bf16 group scale (one per 128 K: the low 16 bits) as an fp16 pair
             const __half hs = __float2half_rn(bf16_bits_to_f32(sbits & 0xffffu));

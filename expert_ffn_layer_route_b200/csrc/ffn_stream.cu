@@ -869,7 +869,11 @@ cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers&
     }
     a.tmem_alloc = alloc;
   }
-  // tensor maps
+  // tensor maps (MOE_W_PROMO=0|64|128|256: the L2 promotion of the weight
+  // boxes, for measuring the DRAM traffic of rows whose 128-byte boxes do
+  // not start on 128-byte lines)
+  int w_promo = 256;
+  if (const char* e = getenv("MOE_W_PROMO")) w_promo = atoi(e);
   const uint64_t row_bytes = (F == kBF16) ? (uint64_t)a.K * 2 : (uint64_t)a.K / 2;
   const uint64_t wrows = gate_up ? 2 * (uint64_t)a.N : (uint64_t)a.N;
   const uint32_t box_rows = (gate_up && half) ? 64u : (uint32_t)kBoxRows;  // rows per weight box
@@ -877,7 +881,7 @@ cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers&
     const uint64_t dims[3] = {row_bytes, wrows, (uint64_t)a.n_phys};
     const uint64_t strides[2] = {row_bytes, (uint64_t)p.stride_w};
     const uint32_t box[3] = {kLine, box_rows, 1};
-    if (!encode_tmap_u8(&a.tm_w, p.w, 3, dims, strides, box, true)) {
+    if (!encode_tmap_u8(&a.tm_w, p.w, 3, dims, strides, box, true, w_promo)) {
       *unsupported = 1;
       return cudaSuccess;
     }
@@ -886,7 +890,7 @@ cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers&
     const uint64_t dims[3] = {row_bytes, wrows, (uint64_t)a.n_shared};
     const uint64_t strides[2] = {row_bytes, (uint64_t)p.stride_w_sh};
     const uint32_t box[3] = {kLine, box_rows, 1};
-    if (!encode_tmap_u8(&a.tm_wsh, p.w_sh, 3, dims, strides, box, true)) {
+    if (!encode_tmap_u8(&a.tm_wsh, p.w_sh, 3, dims, strides, box, true, w_promo)) {
       *unsupported = 1;
       return cudaSuccess;
     }

@@ -37,7 +37,7 @@ uintptr_t current_ctx() {
 }
 
 bool encode_tmap_u8(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
-                    const uint32_t* box, bool swizzle128) {
+                    const uint32_t* box, bool swizzle128, int l2_promo) {
   auto fn = get_encoder();
   if (!fn) return false;
   cuuint64_t gd[5], gs[4];
@@ -51,7 +51,11 @@ bool encode_tmap_u8(CUtensorMap* map, const void* base, int rank, const uint64_t
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE,
                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  l2_promo == 0    ? CU_TENSOR_MAP_L2_PROMOTION_NONE
+                  : l2_promo == 64  ? CU_TENSOR_MAP_L2_PROMOTION_L2_64B
+                  : l2_promo == 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
+                                    : CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 

@@ -9,9 +9,11 @@
 namespace moe {
 
 // Encode a tiled tensor map over bytes (uint8 elements).  dims/strides in
-// bytes; strides[i] is the stride of dimension i+1.  Returns false on failure.
+// bytes; strides[i] is the stride of dimension i+1.  l2_promo: the L2 fetch
+// size the copies are promoted to (0 none, 64, 128 or 256 bytes; default 256).
+// Returns false on failure.
 bool encode_tmap_u8(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
-                    const uint32_t* box, bool swizzle128);
+                    const uint32_t* box, bool swizzle128, int l2_promo = 256);
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar,
                                             uint64_t policy) {

@@ -17,7 +17,10 @@ Per layer l of one decode step:
      their prefetch (copies overlap this layer's FFN on the cache's stream);
   3. read the need set; in waves of at most slots_per_layer experts:
      moe_cache_lookup -> moe_grouped_ffn through the slot map -> release;
-  4. combine; x_{l+1} = x_l + out_l (residual, no norm).
+  4. combine; x_{l+1} = x_l + out_l (residual).
+Each layer's input is the hidden state scaled to unit RMS per token (a
+pre-norm without learned weights): without it the stack's residual stream,
+fed through 48 random SwiGLU layers, grows until it overflows.
 """
 from __future__ import annotations
 
@@ -135,17 +138,20 @@ class OffloadedBank:
         N.moe_combine(d, self.y, self.inv, self.gw, None, out, st)
 
     def decode_step(self, x0: torch.Tensor, prefetch: bool = True, keep: bool = False):
-        """All layers on one batch: x_{l+1} = x_l + out_l.  Returns the last hidden state
-        (and every layer's input and output when keep=True)."""
+        """All layers on one batch: x_{l+1} = x_l + out_l, layer l applied to x_l
+        scaled to unit RMS per token.  Returns the last hidden state (and every
+        layer's input and output when keep=True)."""
         x = x0
         ins, outs = [], []
         for l in range(self.L):
+            xf = x.float()
+            xin = (xf * torch.rsqrt(xf.pow(2).mean(dim=1, keepdim=True) + 1e-6)).to(torch.bfloat16)
             out = torch.empty_like(x)
-            self.forward_layer(l, x, out, prefetch=prefetch)
+            self.forward_layer(l, xin, out, prefetch=prefetch)
             if keep:
-                ins.append(x)
+                ins.append(xin)
                 outs.append(out)
-            x = (x.float() + out.float()).to(torch.bfloat16)
+            x = (xf + out.float()).to(torch.bfloat16)
         return (x, ins, outs) if keep else x
 
     def stats(self) -> dict:

@@ -71,9 +71,11 @@ MIXTRAL = LayerShape("mixtral_prefill", 4096, 8, 2, 14336, "bf16")
 KIMI = LayerShape("kimi_decode", 7168, 384, 8, 2048, "int4", n_shared=1, zipf_s=1.1)
 BANK = LayerShape("offload_bank", 4096, 256, 8, 1536, "nvfp4", zipf_s=1.1)
 
-# The Mixtral-shaped prefill layer with MXFP4 experts (4-bit prefill on the
-# tensor cores); not one of the five measured configurations above.
+# The Mixtral-shaped prefill layer with 4-bit experts (4-bit prefill on the
+# tensor cores); not among the five measured configurations above.
 MIXTRAL_MXFP4 = MIXTRAL.replace(name="mixtral_prefill_mxfp4", wdtype="mxfp4")
+MIXTRAL_NVFP4 = MIXTRAL.replace(name="mixtral_prefill_nvfp4", wdtype="nvfp4")
+MIXTRAL_INT4 = MIXTRAL.replace(name="mixtral_prefill_int4", wdtype="int4")
 
 CONFIG_TOKENS = {
     "tiny": (16,),
@@ -86,7 +88,7 @@ BANK_LAYERS = 48
 BANK_SLOTS_PER_LAYER = 64  # 25% of 256 experts
 BANK_STEPS = 512
 
-CONFIGS = {c.name: c for c in (TINY, GPTOSS, MIXTRAL, KIMI, BANK, MIXTRAL_MXFP4)}
+CONFIGS = {c.name: c for c in (TINY, GPTOSS, MIXTRAL, KIMI, BANK, MIXTRAL_MXFP4, MIXTRAL_NVFP4, MIXTRAL_INT4)}
 
 
 def _gen(seed: int, device) -> torch.Generator:
