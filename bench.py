@@ -569,12 +569,27 @@ def run_offload(args):
         st1 = bank.stats()
         return e0.elapsed_time(e1), {k: st1[k] - st0[k] for k in st1}
 
+    sweep = None
+    if args.bank_prefetch_sweep:
+        # short runs over the prefetch depth (experts prefetched per token), same bank
+        sweep = []
+        first = args.warmup
+        for p_top in [int(v) for v in args.bank_prefetch_sweep.split(",")]:
+            bank.prefetch_top = p_top
+            n_sw = args.bank_sweep_steps
+            ms_sw, d_sw = timed(n_sw, first, p_top > 0)
+            first += n_sw
+            sweep.append({"prefetch_top": p_top, "steps": n_sw, "tokens_per_s": T * n_sw / (ms_sw * 1e-3),
+                          "ms_per_layer": ms_sw / n_sw / L, "hit_rate": d_sw["hits"] / max(d_sw["lookups"], 1),
+                          "bytes_h2d_per_step": d_sw["bytes_h2d"] / n_sw,
+                          "prefetch_used_frac": d_sw["prefetch_used"] / max(d_sw["prefetch_issued"], 1)})
+    bank.prefetch_top = args.bank_prefetch_top if args.bank_prefetch_top >= 0 else shape.top_k
     clocks = ClockSampler()
     clocks.start()
     time.sleep(0.3)
-    ms, d = timed(args.steps, args.warmup, True)
+    ms, d = timed(args.steps, args.warmup + (sum(e["steps"] for e in sweep) if sweep else 0), True)
     n_np = args.bank_noprefetch_steps
-    ms_np, d_np = timed(n_np, args.warmup + args.steps, False) if n_np > 0 else (None, None)
+    ms_np, d_np = timed(n_np, 10 ** 6, False) if n_np > 0 else (None, None)
     clk = clocks.stop()
     h2d = d["bytes_h2d"] / (ms * 1e-3) / 1e9
     per_layer = ms / args.steps / L
@@ -594,7 +609,9 @@ def run_offload(args):
                     "prefetch_used": d["prefetch_used"], "bytes_h2d_per_step": d["bytes_h2d"] / args.steps,
                     "copy_ms_per_step": d["copy_ms"] / args.steps, "h2d_gbs": h2d,
                     "ms_per_layer": per_layer, "resident_ms_per_layer": resident_ms,
-                    "exposed_ms_per_layer": per_layer - resident_ms if resident_ms is not None else None},
+                    "exposed_ms_per_layer": per_layer - resident_ms if resident_ms is not None else None,
+                    "prefetch_top": bank.prefetch_top},
+        "prefetch_sweep": sweep,
         "clocks": clk,
     }
     if ms_np is not None:
@@ -700,6 +717,11 @@ def main():
     ap.add_argument("--bank-layers", type=int, default=mi.BANK_LAYERS, help="layers of the offloaded bank (of 48)")
     ap.add_argument("--bank-noprefetch-steps", type=int, default=16,
                     help="offload_bank: steps of a second run without prefetch (0: none)")
+    ap.add_argument("--bank-prefetch-top", type=int, default=-1,
+                    help="offload_bank: experts prefetched per token (its most likely ones; -1: all top-k)")
+    ap.add_argument("--bank-prefetch-sweep", default="",
+                    help="offload_bank: comma-separated prefetch depths timed first, --bank-sweep-steps each")
+    ap.add_argument("--bank-sweep-steps", type=int, default=48)
     ap.add_argument("--verify-seqs", type=int, default=16, help="verify: sequences per call")
     ap.add_argument("--verify-depth", type=int, default=3, help="verify: drafted tokens per sequence")
     ap.add_argument("--verify-rho", type=float, default=0.5, help="verify: correlation of a sequence's positions")

@@ -25,17 +25,19 @@
 //          significant bits, exact for s in [2^-17, 2^13)) against the same
 //          scaled fp16 activation rows.
 //
-// CTA = 14 warps, one CTA per SM, persistent over tiles of (expert, 256
+// CTA = 22 warps, one CTA per SM, persistent over tiles of (expert, 256
 // activation rows, 256 weight rows); activation rows fastest inside an expert
 // so that CTAs running side by side share each weight tile through L2:
 //   warp 0 (one lane): TMA loads per 64-wide K step into a 3-stage ring: the
 //                      two 128-row activation boxes (128-byte swizzle), the
 //                      256 weight rows' codes (32 bytes each) and their
 //                      16-byte block-scale segments;
-//   warps 6-13       : converters, one weight row per thread: decode the
-//                      row's 64 codes with its scales into 128 bytes of
-//                      16-bit values, written in the 128-byte-swizzled
-//                      K-major layout the MMA reads, into a 2-slot ring;
+//   warps 6-21       : converters, two threads per weight row: each decodes
+//                      32 of the row's 64 codes with their scales into 64
+//                      bytes of 16-bit values (byte-permute table lookups,
+//                      no conversion instructions), written in the
+//                      128-byte-swizzled K-major layout the MMA reads, into
+//                      a 2-slot ring;
 //   warp 1 (one lane): tcgen05.mma (M=128, N=256, K=16), one per 128-row
 //                      activation half, into 2 x 256 TMEM columns; warp 1
 //                      also allocates and frees the 512 columns;
@@ -64,7 +66,7 @@ constexpr int kQCodeBytes = kQBN * 32;    // 256 rows x 64 codes
 constexpr int kQScaleBytes = kQBN * 16;   // 256 rows x one 16-byte scale segment
 constexpr int kQStageBytes = 2 * kQABytes + kQCodeBytes + kQScaleBytes;
 constexpr int kQSlotBytes = kQBN * 128;   // decoded: 256 rows x 64 values x 2 bytes
-constexpr int kQConvWarps = 8;
+constexpr int kQConvWarps = 16;
 constexpr int kQThreads = (6 + kQConvWarps) * 32;
 constexpr int kQMaxGroups = 1024 + 64;
 
@@ -424,15 +426,15 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
         if (kGateUp) {
           __nv_bfloat16* o = a.out_routed + (int64_t)(ti.xrow0 + m) * a.N + ti.n_idx * 128;
 #pragma unroll 1
-          for (int j0 = 0; j0 < 128; j0 += 32) {
-            uint32_t gv[32], uv[32];
-            tc::ld_32x32b_x32(taddr + j0, gv);
-            tc::ld_32x32b_x32(taddr + 128 + j0, uv);
+          for (int j0 = 0; j0 < 128; j0 += 16) {
+            uint32_t gv[16], uv[16];
+            tc::ld_32x32b_x16(taddr + j0, gv);
+            tc::ld_32x32b_x16(taddr + 128 + j0, uv);
             tc::ld_wait();
             if (valid) {
-              uint32_t packed[16];
+              uint32_t packed[8];
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
+              for (int j = 0; j < 8; ++j) {
                 const float g0 = __uint_as_float(gv[2 * j]) * f, g1 = __uint_as_float(gv[2 * j + 1]) * f;
                 const float u0 = __uint_as_float(uv[2 * j]) * f, u1 = __uint_as_float(uv[2 * j + 1]) * f;
                 const float hh0 = g0 / (1.f + __expf(-g0)) * u0;
@@ -441,9 +443,8 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
                 packed[j] = *reinterpret_cast<uint32_t*>(&hb);
               }
               uint4* dst = reinterpret_cast<uint4*>(o + j0);
-#pragma unroll
-              for (int v = 0; v < 4; ++v)
-                dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+              dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+              dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
             }
           }
         } else {
@@ -451,22 +452,21 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
                                                 : a.out_routed + (int64_t)(ti.xrow0 + m) * a.N;
           o += ti.n_idx * kQBN;
 #pragma unroll 1
-          for (int j0 = 0; j0 < kQBN; j0 += 32) {
-            uint32_t v[32];
-            tc::ld_32x32b_x32(taddr + j0, v);
+          for (int j0 = 0; j0 < kQBN; j0 += 16) {
+            uint32_t v[16];
+            tc::ld_32x32b_x16(taddr + j0, v);
             tc::ld_wait();
             if (valid) {
-              uint32_t packed[16];
+              uint32_t packed[8];
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
+              for (int j = 0; j < 8; ++j) {
                 __nv_bfloat162 hb =
                     __floats2bfloat162_rn(__uint_as_float(v[2 * j]) * f, __uint_as_float(v[2 * j + 1]) * f);
                 packed[j] = *reinterpret_cast<uint32_t*>(&hb);
               }
               uint4* dst = reinterpret_cast<uint4*>(o + j0);
-#pragma unroll
-              for (int w = 0; w < 4; ++w)
-                dst[w] = make_uint4(packed[4 * w], packed[4 * w + 1], packed[4 * w + 2], packed[4 * w + 3]);
+              dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+              dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
             }
           }
         }
@@ -477,11 +477,14 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
     }
   } else {
     // ============================================================== converters
-    const int row = tid - 6 * 32;  // weight row of the tile (0..255)
+    // Two threads per weight row: thread `half` decodes K = 32 half .. 32 half + 31
+    // of the step (granules 4 half .. 4 half + 3), one 16-byte code segment;
+    // the 8 threads of a quarter-warp read 4 rows' 128 contiguous code bytes
+    // and write 8 distinct swizzled granule positions.
+    const int cv = tid - 6 * 32;
+    const int row = cv >> 1;  // weight row of the tile (0..255)
+    const int half = cv & 1;
     uint32_t cnt = 0, dcnt = 0;
-    // 16-byte halves of the row's 32 code bytes, read in an order that keeps
-    // the 8 rows of each quarter-warp on distinct banks
-    const int hfirst = (row >> 2) & 1;
     const uint32_t sw = (uint32_t)(row & 7);
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
       for (int ks = 0; ks < ksteps; ++ks) {
@@ -493,43 +496,47 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
           break;
         }
         const uint32_t st = smem_u32(stages + s * kQStageBytes);
-        const uint32_t ca = st + 2 * kQABytes + row * 32;
-        const uint4 c0 = lds128(ca + 16 * hfirst);
-        const uint4 c1 = lds128(ca + 16 * (hfirst ^ 1));
-        const uint32_t cw[8] = {hfirst ? c1.x : c0.x, hfirst ? c1.y : c0.y, hfirst ? c1.z : c0.z,
-                                hfirst ? c1.w : c0.w, hfirst ? c0.x : c1.x, hfirst ? c0.y : c1.y,
-                                hfirst ? c0.z : c1.z, hfirst ? c0.w : c1.w};
+        const uint4 c = lds128(st + 2 * kQABytes + row * 32 + 16 * half);
+        const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
         // this step's scale bytes of the row: at byte (ks*64/blk*sbytes) mod 16 of its segment
         const int soff = ((ks * kQBK / Fm::blk) * Fm::sbytes) & 15;
         const uint32_t sword = lds32(st + 2 * kQABytes + kQCodeBytes + row * 16 + (soff & ~3));
         const uint32_t sbits = sword >> (8 * (soff & 3));
+        // the scale pair(s) of this thread's granules
+        uint32_t s2a = 0, s2b = 0;
+        if constexpr (F == kMXFP4) {
+          // E8M0 of the 32-block `half`, as a bf16 pair (E2M1 x 2^(e-127) is exact in bf16)
+          s2a = e8m0_to_bf16x2((sbits >> (8 * half)) & 0xffu);
+        } else if constexpr (F == kNVFP4) {
+          // E4M3 of the 16-blocks 2 half and 2 half + 1, as fp16 pairs
+          const uint32_t e0 = (sbits >> (16 * half)) & 0xffu, e1 = (sbits >> (16 * half + 8)) & 0xffu;
+          s2a = e4m3x2_to_f16x2(e0 | (e0 << 8));
+          s2b = e4m3x2_to_f16x2(e1 | (e1 << 8));
+        } else {
+          // bf16 group scale (one per 128 K: the low 16 bits) as an fp16 pair
+          const __half2 hs2 = __half2half2(__float2half_rn(bf16_bits_to_f32(sbits & 0xffffu)));
+          s2a = *reinterpret_cast<const uint32_t*>(&hs2);
+        }
         const uint32_t dst = smem_u32(slots + j * kQSlotBytes) + row * 128;
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {  // granule g: K = 8g .. 8g+7 of the step
+        for (int i = 0; i < 4; ++i) {  // granule g = 4 half + i: K = 8g .. 8g+7 of the step
+          const uint32_t g = (uint32_t)(4 * half + i);
           uint32_t o[4];
           if constexpr (F == kMXFP4) {
-            // E8M0 byte of the 32-block holding this granule, as a bf16 pair;
-            // E2M1 x 2^(e-127) is exact in bf16
-            const uint32_t s2 = e8m0_to_bf16x2((sbits >> (8 * (g >> 2))) & 0xffu);
-            e2m1x8_to_16x8_lut<true>(cw[g], o);
+            e2m1x8_to_16x8_lut<true>(cw[i], o);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) o[q] = hmul2_bf16_u32(o[q], s2);
+            for (int q = 0; q < 4; ++q) o[q] = hmul2_bf16_u32(o[q], s2a);
           } else if constexpr (F == kNVFP4) {
-            // E4M3 byte of the 16-block holding this granule, as an fp16 pair
-            const uint32_t e = (sbits >> (8 * (g >> 1))) & 0xffu;
-            const uint32_t s2 = e4m3x2_to_f16x2(e | (e << 8));
-            e2m1x8_to_16x8_lut<false>(cw[g], o);
+            e2m1x8_to_16x8_lut<false>(cw[i], o);
+            const uint32_t s2 = i < 2 ? s2a : s2b;
 #pragma unroll
             for (int q = 0; q < 4; ++q) o[q] = hmul2_u32(o[q], s2);
           } else {
-            // bf16 group scale (one per 128 K: the low 16 bits) as an fp16 pair
-            const __half hs = __float2half_rn(bf16_bits_to_f32(sbits & 0xffffu));
-            const __half2 hs2 = __half2half2(hs);
-            int4x8_to_f16x8_scaled(cw[g], *reinterpret_cast<const uint32_t*>(&hs2), o);
+            int4x8_to_f16x8_scaled(cw[i], s2a, o);
           }
           // 128-byte swizzle: granule g of row r sits at granule g ^ (r & 7)
-          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst + (((uint32_t)g ^ sw) << 4)), "r"(o[0]),
-                       "r"(o[1]), "r"(o[2]), "r"(o[3])
+          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst + ((g ^ sw) << 4)), "r"(o[0]), "r"(o[1]),
+                       "r"(o[2]), "r"(o[3])
                        : "memory");
         }
         fence_proxy_async_smem();  // the MMA (async proxy) reads what these threads wrote

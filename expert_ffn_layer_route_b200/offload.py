@@ -14,7 +14,8 @@ copy per layer).
 Per layer l of one decode step:
   1. route x_l with layer l's router (moe_route_topk) and permute;
   2. predict layer l+1's experts from x_l with layer l+1's router and issue
-     their prefetch (copies overlap this layer's FFN on the cache's stream);
+     the prefetch of each token's `prefetch_top` most likely ones (copies
+     overlap this layer's FFN on the cache's stream);
   3. read the need set; in waves of at most slots_per_layer experts:
      moe_cache_lookup -> moe_grouped_ffn through the slot map -> release;
   4. combine; x_{l+1} = x_l + out_l (residual).
@@ -79,6 +80,12 @@ class OffloadedBank:
         self.y = torch.empty(T * k, d, dtype=torch.bfloat16, device=self.dev)
         self.slot_map = torch.full((E,), -1, dtype=torch.int32, device=self.dev)
         self.trace: List[tuple] = []
+        # experts prefetched per token: its prefetch_top highest-scoring
+        # predictions for the next layer (the whole predicted top-k when
+        # >= top_k; 0 disables prefetch).  Prefetching every prediction fills
+        # the next layer's slots when its need set exceeds them, evicting
+        # experts it was about to use.
+        self.prefetch_top = shape.top_k
 
     # -------------------------------------------------------------- filling
     def fill_layer(self, l: int, layer: Dict[str, object]):
@@ -121,10 +128,11 @@ class OffloadedBank:
         d = self.desc
         N.moe_route_topk(d, x, self.routers[l], self.biases[l], self.idx, self.gw, self.ws, st)
         N.moe_permute(d, self.idx, self.offs, self.rtok, self.inv, st)
-        if prefetch and l + 1 < self.L:
+        if prefetch and self.prefetch_top > 0 and l + 1 < self.L:
             N.moe_route_topk(d, x, self.routers[l + 1], self.biases[l + 1], self.idx_pred, self.gw_pred,
                              self.ws_pred, st)
-            pred = np.unique(self.idx_pred.cpu().numpy())
+            # each token's selection is in descending logit order
+            pred = np.unique(self.idx_pred[:, : self.prefetch_top].cpu().numpy())
             self.trace.append(("prefetch", l + 1, pred.tolist()))
             self.cache.prefetch(l + 1, pred)
         need = np.unique(self.idx.cpu().numpy()).tolist()
