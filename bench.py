@@ -583,7 +583,7 @@ def run_offload(args):
                           "ms_per_layer": ms_sw / n_sw / L, "hit_rate": d_sw["hits"] / max(d_sw["lookups"], 1),
                           "bytes_h2d_per_step": d_sw["bytes_h2d"] / n_sw,
                           "prefetch_used_frac": d_sw["prefetch_used"] / max(d_sw["prefetch_issued"], 1)})
-    bank.prefetch_top = args.bank_prefetch_top if args.bank_prefetch_top >= 0 else shape.top_k
+    bank.prefetch_top = args.bank_prefetch_top if args.bank_prefetch_top >= 0 else None
     clocks = ClockSampler()
     clocks.start()
     time.sleep(0.3)
@@ -610,7 +610,7 @@ def run_offload(args):
                     "copy_ms_per_step": d["copy_ms"] / args.steps, "h2d_gbs": h2d,
                     "ms_per_layer": per_layer, "resident_ms_per_layer": resident_ms,
                     "exposed_ms_per_layer": per_layer - resident_ms if resident_ms is not None else None,
-                    "prefetch_top": bank.prefetch_top},
+                    "prefetch_top": bank.prefetch_top if bank.prefetch_top is not None else "auto"},
         "prefetch_sweep": sweep,
         "clocks": clk,
     }
@@ -718,7 +718,8 @@ def main():
     ap.add_argument("--bank-noprefetch-steps", type=int, default=16,
                     help="offload_bank: steps of a second run without prefetch (0: none)")
     ap.add_argument("--bank-prefetch-top", type=int, default=-1,
-                    help="offload_bank: experts prefetched per token (its most likely ones; -1: all top-k)")
+                    help="offload_bank: experts prefetched per token (its most likely ones; -1: the driver's "
+                         "choice, every prediction when they fit a quarter of the slots, else one)")
     ap.add_argument("--bank-prefetch-sweep", default="",
                     help="offload_bank: comma-separated prefetch depths timed first, --bank-sweep-steps each")
     ap.add_argument("--bank-sweep-steps", type=int, default=48)

@@ -10,9 +10,9 @@
 // the weights are decoded once per tile into 16-bit values in shared memory
 // and fed to tcgen05.mma kind::f16, with fp32 accumulation in tensor memory.
 //
-//   stage 1: D = X_e [256 x K] * [W_gate rows n0..n0+127 ; W_up rows n0..n0+127]^T,
-//            h = silu(D[:, :128]) * D[:, 128:]
-//   stage 2: y = H_e [256 x K] * W_down[n0..n0+255]^T
+//   stage 1: D = X_e [256 x K] * [W_gate rows n0..n0+63 ; W_up rows n0..n0+63]^T,
+//            h = silu(D[:, :64]) * D[:, 64:]
+//   stage 2: y = H_e [256 x K] * W_down[n0..n0+127]^T
 //
 // Operand types, chosen so that every decoded weight is exact:
 //   MXFP4: E2M1 x 2^(s-127) in bf16 (2 significant bits, bf16's exponent
@@ -25,22 +25,24 @@
 //          significant bits, exact for s in [2^-17, 2^13)) against the same
 //          scaled fp16 activation rows.
 //
-// CTA = 22 warps, one CTA per SM, persistent over tiles of (expert, 256
-// activation rows, 256 weight rows); activation rows fastest inside an expert
+// CTA = 14 warps, one CTA per SM, persistent over tiles of (expert, 256
+// activation rows, 128 weight rows); activation rows fastest inside an expert
 // so that CTAs running side by side share each weight tile through L2:
-//   warp 0 (one lane): TMA loads per 64-wide K step into a 3-stage ring: the
+//   warp 0 (one lane): TMA loads per 64-wide K step into a 4-stage ring: the
 //                      two 128-row activation boxes (128-byte swizzle), the
-//                      256 weight rows' codes (32 bytes each) and their
+//                      128 weight rows' codes (32 bytes each) and their
 //                      16-byte block-scale segments;
-//   warps 6-21       : converters, two threads per weight row: each decodes
+//   warps 6-13       : converters, two threads per weight row: each decodes
 //                      32 of the row's 64 codes with their scales into 64
 //                      bytes of 16-bit values (byte-permute table lookups,
 //                      no conversion instructions), written in the
 //                      128-byte-swizzled K-major layout the MMA reads, into
-//                      a 2-slot ring;
-//   warp 1 (one lane): tcgen05.mma (M=128, N=256, K=16), one per 128-row
-//                      activation half, into 2 x 256 TMEM columns; warp 1
-//                      also allocates and frees the 512 columns;
+//                      a 4-slot ring;
+//   warp 1 (one lane): tcgen05.mma (M=128, N=128, K=16), one per 128-row
+//                      activation half, into one of two 2 x 128-column TMEM
+//                      accumulators (so that a tile's epilogue overlaps the
+//                      next tile's MMAs); warp 1 also allocates and frees the
+//                      512 columns;
 //   warps 2-5        : epilogue, one TMEM lane (= activation row) per thread:
 //                      tcgen05.ld, scale, SwiGLU / conversion, bf16 stores.
 // Every wait is bounded (2 s); on expiry the CTA records MOE_ERR_TIMEOUT,
@@ -57,16 +59,16 @@ namespace moe {
 namespace {
 
 constexpr int kQBM = 128;                 // activation rows per MMA (one TMEM lane each)
-constexpr int kQBN = 256;                 // weight rows per tile
+constexpr int kQBN = 128;                 // weight rows per tile
 constexpr int kQBK = 64;                  // K per ring stage (128 bytes of 16-bit values)
-constexpr int kQStages = 3;
-constexpr int kQSlots = 2;                // decoded weight tiles in flight
+constexpr int kQStages = 4;
+constexpr int kQSlots = 4;                // decoded weight tiles in flight
 constexpr int kQABytes = kQBM * 128;      // one activation box
-constexpr int kQCodeBytes = kQBN * 32;    // 256 rows x 64 codes
-constexpr int kQScaleBytes = kQBN * 16;   // 256 rows x one 16-byte scale segment
+constexpr int kQCodeBytes = kQBN * 32;    // 128 rows x 64 codes
+constexpr int kQScaleBytes = kQBN * 16;   // 128 rows x one 16-byte scale segment
 constexpr int kQStageBytes = 2 * kQABytes + kQCodeBytes + kQScaleBytes;
-constexpr int kQSlotBytes = kQBN * 128;   // decoded: 256 rows x 64 values x 2 bytes
-constexpr int kQConvWarps = 16;
+constexpr int kQSlotBytes = kQBN * 128;   // decoded: 128 rows x 64 values x 2 bytes
+constexpr int kQConvWarps = 8;
 constexpr int kQThreads = (6 + kQConvWarps) * 32;
 constexpr int kQMaxGroups = 1024 + 64;
 
@@ -197,16 +199,16 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
   uint64_t* empty = full + kQStages;
   uint64_t* dfull = empty + kQStages;
   uint64_t* dempty = dfull + kQSlots;
-  uint64_t* acc_full = dempty + kQSlots;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* drain = acc_empty + 1;
+  uint64_t* acc_full = dempty + kQSlots;  // [2] accumulator buffers
+  uint64_t* acc_empty = acc_full + 2;     // [2]
+  uint64_t* drain = acc_empty + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_ngroups = reinterpret_cast<int*>(s_tmem + 2);
   int* s_gtile = s_ngroups + 2;                   // [kQMaxGroups + 1] first m-pair of each group (prefix)
   int* s_gexpert = s_gtile + kQMaxGroups + 1;     // [kQMaxGroups] routed expert, or -1 - shared index
 
-  const int n_tiles_n = kGateUp ? a.N / 128 : a.N / kQBN;
+  const int n_tiles_n = kGateUp ? a.N / (kQBN / 2) : a.N / kQBN;
   const int ksteps = a.K / kQBK;
   const int E = a.E;
 
@@ -219,8 +221,10 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
       mbar_init(&dfull[i], kQConvWarps);
       mbar_init(&dempty[i], 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_barrier_init();
@@ -328,8 +332,8 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
         const CUtensorMap* tw = ti.shared_idx >= 0 ? &a.tm_wsh : &a.tm_w;
         const CUtensorMap* ts = ti.shared_idx >= 0 ? &a.tm_ssh : &a.tm_s;
         const int arow = ti.xrow0 + ti.mp * 2 * kQBM;
-        const int n0 = ti.n_idx * (kGateUp ? 128 : kQBN);
-        const int r1 = kGateUp ? a.N + n0 : n0 + 128;  // weight rows of the second box
+        const int n0 = ti.n_idx * (kGateUp ? kQBN / 2 : kQBN);
+        const int r1 = kGateUp ? a.N + n0 : n0 + kQBN / 2;  // weight rows of the second box
         for (int ks = 0; ks < ksteps; ++ks) {
           const int s = cnt % kQStages;
           if (!mbar_wait(&empty[s], ((cnt / kQStages) & 1u) ^ 1u)) {
@@ -364,11 +368,14 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
       for (int t = blockIdx.x; t < total_tiles && !*s_abort; t += gridDim.x, ++i) {
         const QTile ti = decode(t);
         const bool two = ti.n_cols - ti.mp * 2 * kQBM > kQBM;  // second activation half has rows
-        if (!mbar_wait(acc_empty, ((uint32_t)i & 1u) ^ 1u)) {
+        const int buf = i & 1;
+        const uint32_t use = (uint32_t)(i >> 1);
+        if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u)) {
           *s_abort = 1;
           break;
         }
         tc::fence_after_sync();
+        const uint32_t d0 = tmem_base + (uint32_t)(buf * 2 * kQBN);  // this tile's two accumulators
         for (int ks = 0; ks < ksteps; ++ks) {
           const int s = cnt % kQStages;
           const int j = dcnt % kQSlots;
@@ -383,8 +390,8 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
           for (int kk = 0; kk < kQBK / 16; ++kk) {
             const uint64_t bdesc = tc::kmajor_sw128_desc(sb + kk * 32);
             const uint32_t acc = (ks | kk) != 0 ? 1u : 0u;
-            tc::mma_bf16(tmem_base, tc::kmajor_sw128_desc(sa + kk * 32), bdesc, idesc, acc);
-            if (two) tc::mma_bf16(tmem_base + kQBN, tc::kmajor_sw128_desc(sa + kQABytes + kk * 32), bdesc, idesc, acc);
+            tc::mma_bf16(d0, tc::kmajor_sw128_desc(sa + kk * 32), bdesc, idesc, acc);
+            if (two) tc::mma_bf16(d0 + kQBN, tc::kmajor_sw128_desc(sa + kQABytes + kk * 32), bdesc, idesc, acc);
           }
           tc::commit(&empty[s]);   // the activation boxes are free once these MMAs have read them
           tc::commit(&dempty[j]);  // and so is the decoded weight tile
@@ -393,7 +400,7 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
           ++dcnt;
         }
         if (*s_abort) break;
-        tc::commit(acc_full);
+        tc::commit(&acc_full[buf]);
       }
       if (issued) {
         tc::commit(drain);
@@ -406,7 +413,9 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
     const int r = q * 32 + lane;
     int i = 0;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++i) {
-      if (*s_abort || !mbar_wait(acc_full, (uint32_t)i & 1u)) {
+      const int buf = i & 1;
+      const uint32_t use = (uint32_t)(i >> 1);
+      if (*s_abort || !mbar_wait(&acc_full[buf], use & 1u)) {
         *s_abort = 1;
         break;
       }
@@ -422,14 +431,15 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
         if constexpr (!Fm::bf16_ops) {
           if (valid) f = ldexpf(f, __ldg(a.xexp + ti.xrow0 + m));
         }
-        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h2 * kQBN);
+        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 2 * kQBN + h2 * kQBN);
         if (kGateUp) {
-          __nv_bfloat16* o = a.out_routed + (int64_t)(ti.xrow0 + m) * a.N + ti.n_idx * 128;
+          // columns [0, 64): gate rows n0.., [64, 128): up rows of the same outputs
+          __nv_bfloat16* o = a.out_routed + (int64_t)(ti.xrow0 + m) * a.N + ti.n_idx * (kQBN / 2);
 #pragma unroll 1
-          for (int j0 = 0; j0 < 128; j0 += 16) {
+          for (int j0 = 0; j0 < kQBN / 2; j0 += 16) {
             uint32_t gv[16], uv[16];
             tc::ld_32x32b_x16(taddr + j0, gv);
-            tc::ld_32x32b_x16(taddr + 128 + j0, uv);
+            tc::ld_32x32b_x16(taddr + kQBN / 2 + j0, uv);
             tc::ld_wait();
             if (valid) {
               uint32_t packed[8];
@@ -473,7 +483,7 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
       }
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
   } else {
     // ============================================================== converters
@@ -482,7 +492,7 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
     // the 8 threads of a quarter-warp read 4 rows' 128 contiguous code bytes
     // and write 8 distinct swizzled granule positions.
     const int cv = tid - 6 * 32;
-    const int row = cv >> 1;  // weight row of the tile (0..255)
+    const int row = cv >> 1;  // weight row of the tile (0..127)
     const int half = cv & 1;
     uint32_t cnt = 0, dcnt = 0;
     const uint32_t sw = (uint32_t)(row & 7);
@@ -564,7 +574,7 @@ bool gemm_q4_supported(int F, int N, int K, bool gate_up) {
   const int blk = F == kMXFP4 ? 32 : (F == kNVFP4 ? 16 : 128);
   const int sb = F == kINT4 ? 2 : 1;
   if (((K / blk) * sb) % 16) return false;  // TMA row pitch of the scale matrix
-  return gate_up ? (N % 128 == 0) : (N % kQBN == 0);
+  return gate_up ? (N % (kQBN / 2) == 0) : (N % kQBN == 0);
 }
 
 bool gemm_q4_bf16_activations(int F) { return F == kMXFP4; }
@@ -604,10 +614,10 @@ cudaError_t launch_ffn_gemm_q4(int F, bool gate_up, GemmQ4Args a, const GemmQ4Po
                      uint64_t n) {
     const uint64_t wd[3] = {code_row, wrows, n};
     const uint64_t wst[2] = {code_row, (uint64_t)sw};
-    const uint32_t wb[3] = {32, 128, 1};
+    const uint32_t wb[3] = {32, (uint32_t)(kQBN / 2), 1};
     const uint64_t sd[3] = {scale_row, wrows, n};
     const uint64_t sst[2] = {scale_row, (uint64_t)ss};
-    const uint32_t sbx[3] = {16, 128, 1};
+    const uint32_t sbx[3] = {16, (uint32_t)(kQBN / 2), 1};
     return encode_tmap_u8(tw, w, 3, wd, wst, wb, false) && encode_tmap_u8(ts, s, 3, sd, sst, sbx, false);
   };
   ok = ok && weights(&a.tm_w, &a.tm_s, p.w, p.stride_w, p.s, p.stride_s, (uint64_t)a.n_phys);
@@ -621,7 +631,7 @@ cudaError_t launch_ffn_gemm_q4(int F, bool gate_up, GemmQ4Args a, const GemmQ4Po
     *unsupported = 1;
     return cudaSuccess;
   }
-  const int n_tiles_n = gate_up ? a.N / 128 : a.N / kQBN;
+  const int n_tiles_n = gate_up ? a.N / (kQBN / 2) : a.N / kQBN;
   const long rows = (long)a.T * a.k;
   const long max_mp = (rows + 2 * kQBM - 1) / (2 * kQBM) + (a.E < rows ? a.E : rows) +
                       (long)a.n_shared * ((a.T + 2 * kQBM - 1) / (2 * kQBM));
