@@ -584,12 +584,20 @@ def run_offload(args):
                           "bytes_h2d_per_step": d_sw["bytes_h2d"] / n_sw,
                           "prefetch_used_frac": d_sw["prefetch_used"] / max(d_sw["prefetch_issued"], 1)})
     bank.prefetch_top = args.bank_prefetch_top if args.bank_prefetch_top >= 0 else None
+    if args.bank_prefetch_top == -2:
+        bank.prefetch_top = 0
     clocks = ClockSampler()
     clocks.start()
     time.sleep(0.3)
     ms, d = timed(args.steps, args.warmup + (sum(e["steps"] for e in sweep) if sweep else 0), True)
+    # a second run in the same steady state with the other prefetch choice
+    # (every predicted expert when the main run had none, else none)
     n_np = args.bank_noprefetch_steps
-    ms_np, d_np = timed(n_np, 10 ** 6, False) if n_np > 0 else (None, None)
+    main_top = bank.prefetch_top
+    other_top = shape.top_k if main_top == 0 else 0
+    bank.prefetch_top = other_top
+    ms_np, d_np = timed(n_np, 10 ** 6, True) if n_np > 0 else (None, None)
+    bank.prefetch_top = main_top
     clk = clocks.stop()
     h2d = d["bytes_h2d"] / (ms * 1e-3) / 1e9
     per_layer = ms / args.steps / L
@@ -610,15 +618,16 @@ def run_offload(args):
                     "copy_ms_per_step": d["copy_ms"] / args.steps, "h2d_gbs": h2d,
                     "ms_per_layer": per_layer, "resident_ms_per_layer": resident_ms,
                     "exposed_ms_per_layer": per_layer - resident_ms if resident_ms is not None else None,
-                    "prefetch_top": bank.prefetch_top if bank.prefetch_top is not None else "auto"},
+                    "prefetch_top": main_top if main_top is not None else "auto"},
         "prefetch_sweep": sweep,
         "clocks": clk,
     }
     if ms_np is not None:
         pl_np = ms_np / n_np / L
-        line["offload_without_prefetch"] = {
-            "steps": n_np, "ms_per_layer": pl_np, "hit_rate": d_np["hits"] / max(d_np["lookups"], 1),
-            "bytes_h2d_per_step": d_np["bytes_h2d"] / n_np,
+        line["offload_other_prefetch"] = {
+            "prefetch_top": other_top, "steps": n_np, "ms_per_layer": pl_np,
+            "hit_rate": d_np["hits"] / max(d_np["lookups"], 1), "bytes_h2d_per_step": d_np["bytes_h2d"] / n_np,
+            "prefetch_used_frac": d_np["prefetch_used"] / max(d_np["prefetch_issued"], 1),
             "exposed_ms_per_layer": pl_np - resident_ms if resident_ms is not None else None,
             "tokens_per_s": T * n_np / (ms_np * 1e-3)}
     print(json.dumps(line), flush=True)
@@ -715,11 +724,11 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--bank-layers", type=int, default=mi.BANK_LAYERS, help="layers of the offloaded bank (of 48)")
-    ap.add_argument("--bank-noprefetch-steps", type=int, default=16,
-                    help="offload_bank: steps of a second run without prefetch (0: none)")
-    ap.add_argument("--bank-prefetch-top", type=int, default=-1,
-                    help="offload_bank: experts prefetched per token (its most likely ones; -1: the driver's "
-                         "choice, every prediction when they fit a quarter of the slots, else one)")
+    ap.add_argument("--bank-noprefetch-steps", type=int, default=128,
+                    help="offload_bank: steps of a second run with the other prefetch choice (0: none)")
+    ap.add_argument("--bank-prefetch-top", type=int, default=-2,
+                    help="offload_bank: experts prefetched per token, its most likely ones (-2: none, the "
+                         "default; -1: every prediction when they fit a quarter of the slots, else one)")
     ap.add_argument("--bank-prefetch-sweep", default="",
                     help="offload_bank: comma-separated prefetch depths timed first, --bank-sweep-steps each")
     ap.add_argument("--bank-sweep-steps", type=int, default=48)

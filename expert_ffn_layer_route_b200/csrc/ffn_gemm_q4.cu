@@ -10,9 +10,9 @@
 // the weights are decoded once per tile into 16-bit values in shared memory
 // and fed to tcgen05.mma kind::f16, with fp32 accumulation in tensor memory.
 //
-//   stage 1: D = X_e [256 x K] * [W_gate rows n0..n0+63 ; W_up rows n0..n0+63]^T,
-//            h = silu(D[:, :64]) * D[:, 64:]
-//   stage 2: y = H_e [256 x K] * W_down[n0..n0+127]^T
+//   stage 1: D = X_e [256 x K] * [W_gate rows n0..n0+127 ; W_up rows n0..n0+127]^T,
+//            h = silu(D[:, :128]) * D[:, 128:]
+//   stage 2: y = H_e [256 x K] * W_down[n0..n0+255]^T
 //
 // Operand types, chosen so that every decoded weight is exact:
 //   MXFP4: E2M1 x 2^(s-127) in bf16 (2 significant bits, bf16's exponent
@@ -26,23 +26,22 @@
 //          scaled fp16 activation rows.
 //
 // CTA = 14 warps, one CTA per SM, persistent over tiles of (expert, 256
-// activation rows, 128 weight rows); activation rows fastest inside an expert
+// activation rows, 256 weight rows); activation rows fastest inside an expert
 // so that CTAs running side by side share each weight tile through L2:
-//   warp 0 (one lane): TMA loads per 64-wide K step into a 4-stage ring: the
+//   warp 0 (one lane): TMA loads per 64-wide K step into a 3-stage ring: the
 //                      two 128-row activation boxes (128-byte swizzle), the
-//                      128 weight rows' codes (32 bytes each) and their
+//                      256 weight rows' codes (32 bytes each) and their
 //                      16-byte block-scale segments;
-//   warps 6-13       : converters, two threads per weight row: each decodes
-//                      32 of the row's 64 codes with their scales into 64
-//                      bytes of 16-bit values (byte-permute table lookups,
-//                      no conversion instructions), written in the
-//                      128-byte-swizzled K-major layout the MMA reads, into
-//                      a 4-slot ring;
-//   warp 1 (one lane): tcgen05.mma (M=128, N=128, K=16), one per 128-row
-//                      activation half, into one of two 2 x 128-column TMEM
-//                      accumulators (so that a tile's epilogue overlaps the
-//                      next tile's MMAs); warp 1 also allocates and frees the
-//                      512 columns;
+//   warps 6-13       : converters, one weight row per thread: decode the
+//                      row's 64 codes with its scales into 128 bytes of
+//                      16-bit values (NVFP4 and INT4 by byte-permute table
+//                      lookups and 16-bit multiplies, MXFP4 through the
+//                      hardware E2M1 conversion: the fastest measured for
+//                      each), written in the 128-byte-swizzled K-major
+//                      layout the MMA reads, into a 2-slot ring;
+//   warp 1 (one lane): tcgen05.mma (M=128, N=256, K=16), one per 128-row
+//                      activation half, into 2 x 256 TMEM columns; warp 1
+//                      also allocates and frees the 512 columns;
 //   warps 2-5        : epilogue, one TMEM lane (= activation row) per thread:
 //                      tcgen05.ld, scale, SwiGLU / conversion, bf16 stores.
 // Every wait is bounded (2 s); on expiry the CTA records MOE_ERR_TIMEOUT,
@@ -59,15 +58,15 @@ namespace moe {
 namespace {
 
 constexpr int kQBM = 128;                 // activation rows per MMA (one TMEM lane each)
-constexpr int kQBN = 128;                 // weight rows per tile
+constexpr int kQBN = 256;                 // weight rows per tile
 constexpr int kQBK = 64;                  // K per ring stage (128 bytes of 16-bit values)
-constexpr int kQStages = 4;
-constexpr int kQSlots = 4;                // decoded weight tiles in flight
+constexpr int kQStages = 3;
+constexpr int kQSlots = 2;                // decoded weight tiles in flight
 constexpr int kQABytes = kQBM * 128;      // one activation box
-constexpr int kQCodeBytes = kQBN * 32;    // 128 rows x 64 codes
-constexpr int kQScaleBytes = kQBN * 16;   // 128 rows x one 16-byte scale segment
+constexpr int kQCodeBytes = kQBN * 32;    // 256 rows x 64 codes
+constexpr int kQScaleBytes = kQBN * 16;   // 256 rows x one 16-byte scale segment
 constexpr int kQStageBytes = 2 * kQABytes + kQCodeBytes + kQScaleBytes;
-constexpr int kQSlotBytes = kQBN * 128;   // decoded: 128 rows x 64 values x 2 bytes
+constexpr int kQSlotBytes = kQBN * 128;   // decoded: 256 rows x 64 values x 2 bytes
 constexpr int kQConvWarps = 8;
 constexpr int kQThreads = (6 + kQConvWarps) * 32;
 constexpr int kQMaxGroups = 1024 + 64;
@@ -114,35 +113,22 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return r;
 }
 
-// Eight E2M1 codes (nibble i = K i of the word) -> four 16-bit pairs in K
-// order (2i, 2i+1) by table lookup on the integer pipe: byte permutes pick
-// each magnitude's high (and, for bf16, low) byte from 8-entry tables, a
-// second permute interleaves them, and the code's sign bit is moved to bit
-// 15 / 31 of its pair.  Tables: E2M1 magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 as
-// bf16 (0x0000 3F00 3F80 3FC0 4000 4040 4080 40C0) or fp16 (0x0000 3800 3C00
-// 3E00 4000 4200 4400 4600, whose low bytes are all zero).  No conversion
-// instruction is used: the conversion unit's throughput would otherwise bound
-// the converters.
-template <bool kBf16>
-__device__ __forceinline__ void e2m1x8_to_16x8_lut(uint32_t w, uint32_t (&o)[4]) {
+// Eight E2M1 codes (nibble i = K i of the word) -> four fp16 pairs in K order
+// (2i, 2i+1) by table lookup on the integer pipe: a byte permute picks each
+// magnitude's high byte from an 8-entry table (E2M1 magnitudes 0, 0.5, 1,
+// 1.5, 2, 3, 4, 6 are the fp16 values 0x0000 3800 3C00 3E00 4000 4200 4400
+// 4600, whose low bytes are all zero), a second permute spreads them into
+// the pairs, and the code's sign bit is moved to bit 15 / 31 of its pair.
+__device__ __forceinline__ void e2m1x8_to_f16x8_lut(uint32_t w, uint32_t (&o)[4]) {
   const uint32_t m = w & 0x77777777u;  // magnitude codes
   const uint32_t m2 = m >> 16;
   const uint32_t s8 = w & 0x88888888u;  // sign bits
   const uint32_t t = s8 << 4;           // sign of the even code of byte b in the msb of byte b
-  if constexpr (kBf16) {
-    const uint32_t hA = prmt(0x3F3F3F00u, 0x40404040u, m), lA = prmt(0xC0800000u, 0xC0804000u, m);
-    const uint32_t hB = prmt(0x3F3F3F00u, 0x40404040u, m2), lB = prmt(0xC0800000u, 0xC0804000u, m2);
-    o[0] = prmt(lA, hA, 0x5140u);
-    o[1] = prmt(lA, hA, 0x7362u);
-    o[2] = prmt(lB, hB, 0x5140u);
-    o[3] = prmt(lB, hB, 0x7362u);
-  } else {
-    const uint32_t hA = prmt(0x3E3C3800u, 0x46444240u, m), hB = prmt(0x3E3C3800u, 0x46444240u, m2);
-    o[0] = prmt(hA, 0u, 0x1404u);
-    o[1] = prmt(hA, 0u, 0x3424u);
-    o[2] = prmt(hB, 0u, 0x1404u);
-    o[3] = prmt(hB, 0u, 0x3424u);
-  }
+  const uint32_t hA = prmt(0x3E3C3800u, 0x46444240u, m), hB = prmt(0x3E3C3800u, 0x46444240u, m2);
+  o[0] = prmt(hA, 0u, 0x1404u);
+  o[1] = prmt(hA, 0u, 0x3424u);
+  o[2] = prmt(hB, 0u, 0x1404u);
+  o[3] = prmt(hB, 0u, 0x3424u);
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
     // byte 1 <- byte b of t (even code's sign), byte 3 <- byte b of s8 (odd code's sign)
@@ -151,16 +137,13 @@ __device__ __forceinline__ void e2m1x8_to_16x8_lut(uint32_t w, uint32_t (&o)[4])
   }
 }
 
-// bf16 pair (2^(e-127), 2^(e-127)) of an E8M0 scale byte (e = 0: 2^-127, a
-// bf16 subnormal; e = 255: NaN).
-__device__ __forceinline__ uint32_t e8m0_to_bf16x2(uint32_t e) {
-  const uint32_t b = e == 0u ? 0x0040u : (e == 255u ? 0x7fc0u : (e << 7));
-  return b | (b << 16);
-}
-
-__device__ __forceinline__ uint32_t hmul2_bf16_u32(uint32_t a, uint32_t b) {
-  __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
-  return *reinterpret_cast<uint32_t*>(&r);
+// fp16 pair -> bf16 pair after multiplying both by f (exact when the products
+// have at most 8 significant bits and lie in bf16's range).
+__device__ __forceinline__ uint32_t f16x2_scale_to_bf16x2(uint32_t h2, float f) {
+  const __half2 h = *reinterpret_cast<const __half2*>(&h2);
+  const float2 v = __half22float2(h);
+  __nv_bfloat162 b = __floats2bfloat162_rn(v.x * f, v.y * f);
+  return *reinterpret_cast<uint32_t*>(&b);
 }
 
 // Eight INT4 codes (nibble i = K i of the word) -> four fp16 pairs in K order
@@ -199,16 +182,16 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
   uint64_t* empty = full + kQStages;
   uint64_t* dfull = empty + kQStages;
   uint64_t* dempty = dfull + kQSlots;
-  uint64_t* acc_full = dempty + kQSlots;  // [2] accumulator buffers
-  uint64_t* acc_empty = acc_full + 2;     // [2]
-  uint64_t* drain = acc_empty + 2;
+  uint64_t* acc_full = dempty + kQSlots;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_empty + 1;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_ngroups = reinterpret_cast<int*>(s_tmem + 2);
   int* s_gtile = s_ngroups + 2;                   // [kQMaxGroups + 1] first m-pair of each group (prefix)
   int* s_gexpert = s_gtile + kQMaxGroups + 1;     // [kQMaxGroups] routed expert, or -1 - shared index
 
-  const int n_tiles_n = kGateUp ? a.N / (kQBN / 2) : a.N / kQBN;
+  const int n_tiles_n = kGateUp ? a.N / 128 : a.N / kQBN;
   const int ksteps = a.K / kQBK;
   const int E = a.E;
 
@@ -221,10 +204,8 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
       mbar_init(&dfull[i], kQConvWarps);
       mbar_init(&dempty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4);
-    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 4);
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_barrier_init();
@@ -332,8 +313,8 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
         const CUtensorMap* tw = ti.shared_idx >= 0 ? &a.tm_wsh : &a.tm_w;
         const CUtensorMap* ts = ti.shared_idx >= 0 ? &a.tm_ssh : &a.tm_s;
         const int arow = ti.xrow0 + ti.mp * 2 * kQBM;
-        const int n0 = ti.n_idx * (kGateUp ? kQBN / 2 : kQBN);
-        const int r1 = kGateUp ? a.N + n0 : n0 + kQBN / 2;  // weight rows of the second box
+        const int n0 = ti.n_idx * (kGateUp ? 128 : kQBN);
+        const int r1 = kGateUp ? a.N + n0 : n0 + 128;  // weight rows of the second box
         for (int ks = 0; ks < ksteps; ++ks) {
           const int s = cnt % kQStages;
           if (!mbar_wait(&empty[s], ((cnt / kQStages) & 1u) ^ 1u)) {
@@ -368,14 +349,11 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
       for (int t = blockIdx.x; t < total_tiles && !*s_abort; t += gridDim.x, ++i) {
         const QTile ti = decode(t);
         const bool two = ti.n_cols - ti.mp * 2 * kQBM > kQBM;  // second activation half has rows
-        const int buf = i & 1;
-        const uint32_t use = (uint32_t)(i >> 1);
-        if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u)) {
+        if (!mbar_wait(acc_empty, ((uint32_t)i & 1u) ^ 1u)) {
           *s_abort = 1;
           break;
         }
         tc::fence_after_sync();
-        const uint32_t d0 = tmem_base + (uint32_t)(buf * 2 * kQBN);  // this tile's two accumulators
         for (int ks = 0; ks < ksteps; ++ks) {
           const int s = cnt % kQStages;
           const int j = dcnt % kQSlots;
@@ -390,8 +368,8 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
           for (int kk = 0; kk < kQBK / 16; ++kk) {
             const uint64_t bdesc = tc::kmajor_sw128_desc(sb + kk * 32);
             const uint32_t acc = (ks | kk) != 0 ? 1u : 0u;
-            tc::mma_bf16(d0, tc::kmajor_sw128_desc(sa + kk * 32), bdesc, idesc, acc);
-            if (two) tc::mma_bf16(d0 + kQBN, tc::kmajor_sw128_desc(sa + kQABytes + kk * 32), bdesc, idesc, acc);
+            tc::mma_bf16(tmem_base, tc::kmajor_sw128_desc(sa + kk * 32), bdesc, idesc, acc);
+            if (two) tc::mma_bf16(tmem_base + kQBN, tc::kmajor_sw128_desc(sa + kQABytes + kk * 32), bdesc, idesc, acc);
           }
           tc::commit(&empty[s]);   // the activation boxes are free once these MMAs have read them
           tc::commit(&dempty[j]);  // and so is the decoded weight tile
@@ -400,7 +378,7 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
           ++dcnt;
         }
         if (*s_abort) break;
-        tc::commit(&acc_full[buf]);
+        tc::commit(acc_full);
       }
       if (issued) {
         tc::commit(drain);
@@ -413,9 +391,7 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
     const int r = q * 32 + lane;
     int i = 0;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++i) {
-      const int buf = i & 1;
-      const uint32_t use = (uint32_t)(i >> 1);
-      if (*s_abort || !mbar_wait(&acc_full[buf], use & 1u)) {
+      if (*s_abort || !mbar_wait(acc_full, (uint32_t)i & 1u)) {
         *s_abort = 1;
         break;
       }
@@ -431,20 +407,19 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
         if constexpr (!Fm::bf16_ops) {
           if (valid) f = ldexpf(f, __ldg(a.xexp + ti.xrow0 + m));
         }
-        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 2 * kQBN + h2 * kQBN);
+        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h2 * kQBN);
         if (kGateUp) {
-          // columns [0, 64): gate rows n0.., [64, 128): up rows of the same outputs
-          __nv_bfloat16* o = a.out_routed + (int64_t)(ti.xrow0 + m) * a.N + ti.n_idx * (kQBN / 2);
+          __nv_bfloat16* o = a.out_routed + (int64_t)(ti.xrow0 + m) * a.N + ti.n_idx * 128;
 #pragma unroll 1
-          for (int j0 = 0; j0 < kQBN / 2; j0 += 16) {
-            uint32_t gv[16], uv[16];
-            tc::ld_32x32b_x16(taddr + j0, gv);
-            tc::ld_32x32b_x16(taddr + kQBN / 2 + j0, uv);
+          for (int j0 = 0; j0 < 128; j0 += 32) {
+            uint32_t gv[32], uv[32];
+            tc::ld_32x32b_x32(taddr + j0, gv);
+            tc::ld_32x32b_x32(taddr + 128 + j0, uv);
             tc::ld_wait();
             if (valid) {
-              uint32_t packed[8];
+              uint32_t packed[16];
 #pragma unroll
-              for (int j = 0; j < 8; ++j) {
+              for (int j = 0; j < 16; ++j) {
                 const float g0 = __uint_as_float(gv[2 * j]) * f, g1 = __uint_as_float(gv[2 * j + 1]) * f;
                 const float u0 = __uint_as_float(uv[2 * j]) * f, u1 = __uint_as_float(uv[2 * j + 1]) * f;
                 const float hh0 = g0 / (1.f + __expf(-g0)) * u0;
@@ -453,8 +428,9 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
                 packed[j] = *reinterpret_cast<uint32_t*>(&hb);
               }
               uint4* dst = reinterpret_cast<uint4*>(o + j0);
-              dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-              dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
             }
           }
         } else {
@@ -462,39 +438,37 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
                                                 : a.out_routed + (int64_t)(ti.xrow0 + m) * a.N;
           o += ti.n_idx * kQBN;
 #pragma unroll 1
-          for (int j0 = 0; j0 < kQBN; j0 += 16) {
-            uint32_t v[16];
-            tc::ld_32x32b_x16(taddr + j0, v);
+          for (int j0 = 0; j0 < kQBN; j0 += 32) {
+            uint32_t v[32];
+            tc::ld_32x32b_x32(taddr + j0, v);
             tc::ld_wait();
             if (valid) {
-              uint32_t packed[8];
+              uint32_t packed[16];
 #pragma unroll
-              for (int j = 0; j < 8; ++j) {
+              for (int j = 0; j < 16; ++j) {
                 __nv_bfloat162 hb =
                     __floats2bfloat162_rn(__uint_as_float(v[2 * j]) * f, __uint_as_float(v[2 * j + 1]) * f);
                 packed[j] = *reinterpret_cast<uint32_t*>(&hb);
               }
               uint4* dst = reinterpret_cast<uint4*>(o + j0);
-              dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-              dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+#pragma unroll
+              for (int w = 0; w < 4; ++w)
+                dst[w] = make_uint4(packed[4 * w], packed[4 * w + 1], packed[4 * w + 2], packed[4 * w + 3]);
             }
           }
         }
       }
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if (lane == 0) mbar_arrive(acc_empty);
     }
   } else {
     // ============================================================== converters
-    // Two threads per weight row: thread `half` decodes K = 32 half .. 32 half + 31
-    // of the step (granules 4 half .. 4 half + 3), one 16-byte code segment;
-    // the 8 threads of a quarter-warp read 4 rows' 128 contiguous code bytes
-    // and write 8 distinct swizzled granule positions.
-    const int cv = tid - 6 * 32;
-    const int row = cv >> 1;  // weight row of the tile (0..127)
-    const int half = cv & 1;
+    const int row = tid - 6 * 32;  // weight row of the tile (0..255)
     uint32_t cnt = 0, dcnt = 0;
+    // 16-byte halves of the row's 32 code bytes, read in an order that keeps
+    // the 8 rows of each quarter-warp on distinct banks
+    const int hfirst = (row >> 2) & 1;
     const uint32_t sw = (uint32_t)(row & 7);
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
       for (int ks = 0; ks < ksteps; ++ks) {
@@ -506,47 +480,47 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_gemm_q4_kernel(const __grid_
           break;
         }
         const uint32_t st = smem_u32(stages + s * kQStageBytes);
-        const uint4 c = lds128(st + 2 * kQABytes + row * 32 + 16 * half);
-        const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+        const uint32_t ca = st + 2 * kQABytes + row * 32;
+        const uint4 c0 = lds128(ca + 16 * hfirst);
+        const uint4 c1 = lds128(ca + 16 * (hfirst ^ 1));
+        const uint32_t cw[8] = {hfirst ? c1.x : c0.x, hfirst ? c1.y : c0.y, hfirst ? c1.z : c0.z,
+                                hfirst ? c1.w : c0.w, hfirst ? c0.x : c1.x, hfirst ? c0.y : c1.y,
+                                hfirst ? c0.z : c1.z, hfirst ? c0.w : c1.w};
         // this step's scale bytes of the row: at byte (ks*64/blk*sbytes) mod 16 of its segment
         const int soff = ((ks * kQBK / Fm::blk) * Fm::sbytes) & 15;
         const uint32_t sword = lds32(st + 2 * kQABytes + kQCodeBytes + row * 16 + (soff & ~3));
         const uint32_t sbits = sword >> (8 * (soff & 3));
-        // the scale pair(s) of this thread's granules
-        uint32_t s2a = 0, s2b = 0;
-        if constexpr (F == kMXFP4) {
-          // E8M0 of the 32-block `half`, as a bf16 pair (E2M1 x 2^(e-127) is exact in bf16)
-          s2a = e8m0_to_bf16x2((sbits >> (8 * half)) & 0xffu);
-        } else if constexpr (F == kNVFP4) {
-          // E4M3 of the 16-blocks 2 half and 2 half + 1, as fp16 pairs
-          const uint32_t e0 = (sbits >> (16 * half)) & 0xffu, e1 = (sbits >> (16 * half + 8)) & 0xffu;
-          s2a = e4m3x2_to_f16x2(e0 | (e0 << 8));
-          s2b = e4m3x2_to_f16x2(e1 | (e1 << 8));
-        } else {
-          // bf16 group scale (one per 128 K: the low 16 bits) as an fp16 pair
-          const __half2 hs2 = __half2half2(__float2half_rn(bf16_bits_to_f32(sbits & 0xffffu)));
-          s2a = *reinterpret_cast<const uint32_t*>(&hs2);
-        }
         const uint32_t dst = smem_u32(slots + j * kQSlotBytes) + row * 128;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {  // granule g = 4 half + i: K = 8g .. 8g+7 of the step
-          const uint32_t g = (uint32_t)(4 * half + i);
+        for (int g = 0; g < 8; ++g) {  // granule g: K = 8g .. 8g+7 of the step
           uint32_t o[4];
           if constexpr (F == kMXFP4) {
-            e2m1x8_to_16x8_lut<true>(cw[i], o);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) o[q] = hmul2_bf16_u32(o[q], s2a);
+            // E8M0 scale of the 32-block holding this granule; E2M1 -> fp16 by
+            // the hardware conversion, x 2^(e-127) in fp32, -> bf16 (exact:
+            // 2 significant bits, bf16's exponent range)
+            const float f = e8m0_to_f32((sbits >> (8 * (g >> 2))) & 0xffu);
+            uint32_t h0, h1, h2, h3;
+            e2m1x8_to_f16x8(cw[g], h0, h1, h2, h3);
+            o[0] = f16x2_scale_to_bf16x2(h0, f);
+            o[1] = f16x2_scale_to_bf16x2(h1, f);
+            o[2] = f16x2_scale_to_bf16x2(h2, f);
+            o[3] = f16x2_scale_to_bf16x2(h3, f);
           } else if constexpr (F == kNVFP4) {
-            e2m1x8_to_16x8_lut<false>(cw[i], o);
-            const uint32_t s2 = i < 2 ? s2a : s2b;
+            // E4M3 byte of the 16-block holding this granule, as an fp16 pair
+            const uint32_t e = (sbits >> (8 * (g >> 1))) & 0xffu;
+            const uint32_t s2 = e4m3x2_to_f16x2(e | (e << 8));
+            e2m1x8_to_f16x8_lut(cw[g], o);
 #pragma unroll
             for (int q = 0; q < 4; ++q) o[q] = hmul2_u32(o[q], s2);
           } else {
-            int4x8_to_f16x8_scaled(cw[i], s2a, o);
+            // bf16 group scale (one per 128 K: the low 16 bits) as an fp16 pair
+            const __half hs = __float2half_rn(bf16_bits_to_f32(sbits & 0xffffu));
+            const __half2 hs2 = __half2half2(hs);
+            int4x8_to_f16x8_scaled(cw[g], *reinterpret_cast<const uint32_t*>(&hs2), o);
           }
           // 128-byte swizzle: granule g of row r sits at granule g ^ (r & 7)
-          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst + ((g ^ sw) << 4)), "r"(o[0]), "r"(o[1]),
-                       "r"(o[2]), "r"(o[3])
+          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst + (((uint32_t)g ^ sw) << 4)), "r"(o[0]),
+                       "r"(o[1]), "r"(o[2]), "r"(o[3])
                        : "memory");
         }
         fence_proxy_async_smem();  // the MMA (async proxy) reads what these threads wrote
@@ -574,7 +548,7 @@ bool gemm_q4_supported(int F, int N, int K, bool gate_up) {
   const int blk = F == kMXFP4 ? 32 : (F == kNVFP4 ? 16 : 128);
   const int sb = F == kINT4 ? 2 : 1;
   if (((K / blk) * sb) % 16) return false;  // TMA row pitch of the scale matrix
-  return gate_up ? (N % (kQBN / 2) == 0) : (N % kQBN == 0);
+  return gate_up ? (N % 128 == 0) : (N % kQBN == 0);
 }
 
 bool gemm_q4_bf16_activations(int F) { return F == kMXFP4; }
@@ -614,10 +588,10 @@ cudaError_t launch_ffn_gemm_q4(int F, bool gate_up, GemmQ4Args a, const GemmQ4Po
                      uint64_t n) {
     const uint64_t wd[3] = {code_row, wrows, n};
     const uint64_t wst[2] = {code_row, (uint64_t)sw};
-    const uint32_t wb[3] = {32, (uint32_t)(kQBN / 2), 1};
+    const uint32_t wb[3] = {32, 128, 1};
     const uint64_t sd[3] = {scale_row, wrows, n};
     const uint64_t sst[2] = {scale_row, (uint64_t)ss};
-    const uint32_t sbx[3] = {16, (uint32_t)(kQBN / 2), 1};
+    const uint32_t sbx[3] = {16, 128, 1};
     return encode_tmap_u8(tw, w, 3, wd, wst, wb, false) && encode_tmap_u8(ts, s, 3, sd, sst, sbx, false);
   };
   ok = ok && weights(&a.tm_w, &a.tm_s, p.w, p.stride_w, p.s, p.stride_s, (uint64_t)a.n_phys);
@@ -631,7 +605,7 @@ cudaError_t launch_ffn_gemm_q4(int F, bool gate_up, GemmQ4Args a, const GemmQ4Po
     *unsupported = 1;
     return cudaSuccess;
   }
-  const int n_tiles_n = gate_up ? a.N / (kQBN / 2) : a.N / kQBN;
+  const int n_tiles_n = gate_up ? a.N / 128 : a.N / kQBN;
   const long rows = (long)a.T * a.k;
   const long max_mp = (rows + 2 * kQBM - 1) / (2 * kQBM) + (a.E < rows ? a.E : rows) +
                       (long)a.n_shared * ((a.T + 2 * kQBM - 1) / (2 * kQBM));

@@ -13,9 +13,9 @@ copy per layer).
 
 Per layer l of one decode step:
   1. route x_l with layer l's router (moe_route_topk) and permute;
-  2. predict layer l+1's experts from x_l with layer l+1's router and issue
-     the prefetch of each token's most likely ones (`prefetch_top`; copies
-     overlap this layer's FFN on the cache's stream);
+  2. optionally (`prefetch_top`), predict layer l+1's experts from x_l with
+     layer l+1's router and issue the prefetch of each token's most likely
+     ones (copies overlap this layer's FFN on the cache's stream);
   3. read the need set; in waves of at most slots_per_layer experts:
      moe_cache_lookup -> moe_grouped_ffn through the slot map -> release;
   4. combine; x_{l+1} = x_l + out_l (residual).
@@ -81,14 +81,17 @@ class OffloadedBank:
         self.slot_map = torch.full((E,), -1, dtype=torch.int32, device=self.dev)
         self.trace: List[tuple] = []
         # experts prefetched per token: its prefetch_top highest-scoring
-        # predictions for the next layer (0 disables prefetch; None chooses:
+        # predictions for the next layer (0: no prefetch, the default; None:
         # every prediction when the predicted set fits in a quarter of the
-        # layer's slots, else each token's most likely one).  Prefetching
-        # every prediction fills the next layer's slots when its need set
-        # exceeds them, evicting experts it was about to use (measured on the
-        # 48-layer bank: at 16 tokens per step it copies 30% more bytes and
-        # runs 20% slower than no prefetch; at one token it is the fastest).
-        self.prefetch_top = None
+        # layer's slots, else each token's most likely one).  Measured on the
+        # 48-layer NVFP4 bank with 25% of the experts resident, in steady
+        # state, the stack is bound by the host-to-device copies at 1, 4 and
+        # 16 tokens per step, and a prefetch hides no copy time: it only adds
+        # the bytes of predictions that go unused (about 17% of them) and
+        # evicts experts the layer was about to use, so no prefetch was faster
+        # at every batch size.  With faster copies or more slots than the need
+        # set the overlap would pay, hence the option.
+        self.prefetch_top = 0
 
     # -------------------------------------------------------------- filling
     def fill_layer(self, l: int, layer: Dict[str, object]):

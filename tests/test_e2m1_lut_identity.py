@@ -1,17 +1,14 @@
-"""The table-lookup E2M1 decode of the 4-bit tensor-core path, checked on the
-CPU in exact arithmetic.
+"""The table-lookup E2M1 decode of the 4-bit tensor-core path (NVFP4
+experts), checked on the CPU in exact arithmetic.
 
 The converter warps turn eight E2M1 codes (one 32-bit word, nibble i = K i)
-into four 16-bit pairs with byte permutes only: magnitudes through 8-entry
-byte tables (bf16: high and low bytes; fp16: high bytes, the low bytes being
-zero), an interleaving permute, and the sign bits moved to bit 15 / 31 of each
-pair.  This test restates those steps (the PTX prmt semantics: bytes 0-3 from
+into four fp16 pairs with byte permutes only: magnitudes through an 8-entry
+byte table of fp16 high bytes (the low bytes being zero), a spreading
+permute, and the sign bits moved to bit 15 / 31 of each pair.  This test restates those steps (the PTX prmt semantics: bytes 0-3 from
 the first operand, 4-7 from the second, selector nibble n picks output byte n)
 and compares every result with the E2M1 value from the format definition,
 for every code in every nibble position.
 """
-import struct
-
 import numpy as np
 
 E2M1 = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
@@ -27,27 +24,20 @@ def prmt(a, b, sel):
     return out
 
 
-def lut_decode(w, bf16):
+def lut_decode(w):
     m = w & 0x77777777
     m2 = m >> 16
     s8 = w & 0x88888888
     t = (s8 << 4) & 0xFFFFFFFF
-    if bf16:
-        hA, lA = prmt(0x3F3F3F00, 0x40404040, m), prmt(0xC0800000, 0xC0804000, m)
-        hB, lB = prmt(0x3F3F3F00, 0x40404040, m2), prmt(0xC0800000, 0xC0804000, m2)
-        o = [prmt(lA, hA, 0x5140), prmt(lA, hA, 0x7362), prmt(lB, hB, 0x5140), prmt(lB, hB, 0x7362)]
-    else:
-        hA, hB = prmt(0x3E3C3800, 0x46444240, m), prmt(0x3E3C3800, 0x46444240, m2)
-        o = [prmt(hA, 0, 0x1404), prmt(hA, 0, 0x3424), prmt(hB, 0, 0x1404), prmt(hB, 0, 0x3424)]
+    hA, hB = prmt(0x3E3C3800, 0x46444240, m), prmt(0x3E3C3800, 0x46444240, m2)
+    o = [prmt(hA, 0, 0x1404), prmt(hA, 0, 0x3424), prmt(hB, 0, 0x1404), prmt(hB, 0, 0x3424)]
     for b in range(4):
         sg = prmt(t, s8, b * 0x11 | (4 + b) * 0x1100)
         o[b] |= sg & 0x80008000
     return o
 
 
-def half_bits_to_float(h, bf16):
-    if bf16:
-        return struct.unpack("<f", struct.pack("<I", h << 16))[0]
+def f16_bits_to_float(h):
     return float(np.array([h], dtype=np.uint16).view(np.float16)[0])
 
 
@@ -56,28 +46,26 @@ def e2m1(code):
     return -v if code & 8 else v
 
 
-def check_word(w, bf16):
-    o = lut_decode(w, bf16)
+def check_word(w):
+    o = lut_decode(w)
     for i in range(8):
         h = (o[i // 2] >> (16 * (i % 2))) & 0xFFFF
-        got = half_bits_to_float(h, bf16)
+        got = f16_bits_to_float(h)
         want = e2m1((w >> (4 * i)) & 0xF)
         assert got == want and (np.signbit(got) == bool((w >> (4 * i + 3)) & 1) or want != 0), (hex(w), i, got, want)
 
 
 def test_every_code_in_every_position():
-    for bf16 in (True, False):
-        for pos in range(8):
-            for code in range(16):
-                for fill in (0x0, 0x9, 0xF, 0x7):
-                    w = 0
-                    for i in range(8):
-                        w |= (code if i == pos else fill) << (4 * i)
-                    check_word(w, bf16)
+    for pos in range(8):
+        for code in range(16):
+            for fill in (0x0, 0x9, 0xF, 0x7):
+                w = 0
+                for i in range(8):
+                    w |= (code if i == pos else fill) << (4 * i)
+                check_word(w)
 
 
 def test_random_words():
     rng = np.random.default_rng(0)
     for w in rng.integers(0, 2 ** 32, size=3000, dtype=np.uint64).tolist():
-        check_word(int(w), True)
-        check_word(int(w), False)
+        check_word(int(w))

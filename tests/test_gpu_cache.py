@@ -38,6 +38,7 @@ def test_cache_outputs_equal_resident_layer_and_trace_replays(fmt, C):
     shape = mi.BANK.replace(d_model=512, d_ff=384 if fmt != "int4" else 256, n_experts=16, top_k=4, wdtype=fmt)
     L, T = 3, 4
     bank, layers = _bank(shape, L, C, T)
+    bank.prefetch_top = shape.top_k  # prefetch every predicted expert (the driver's default is none)
     for step in range(3):
         x0 = mi.bank_step_tokens(step, T, shape.d_model, 5, "cuda")
         _, ins, outs = bank.decode_step(x0, prefetch=True, keep=True)
@@ -51,6 +52,7 @@ def test_cache_outputs_equal_resident_layer_and_trace_replays(fmt, C):
     assert {k: st[k] for k in STAT_KEYS} == r.stats
     for l in range(L):
         assert bank.cache.slot_map(l) == r.slot_map(l)
+    assert st["prefetch_issued"] > 0
     copies = st["misses"] + st["prefetch_issued"]
     assert st["bytes_h2d"] == copies * bank.blob.size
     assert st["copy_ms"] > 0.0
