@@ -355,6 +355,8 @@ Q4_GEMM_CASES = [
     ("mxfp4_gemm_small_groups", mi.GPTOSS.replace(d_model=512, d_ff=512, n_experts=8, top_k=2), 290),
     ("nvfp4_gemm", mi.BANK.replace(d_model=512, d_ff=768, n_experts=6, top_k=2), 400),
     ("int4_gemm_shared", mi.KIMI.replace(d_model=1024, d_ff=1024, n_experts=8, top_k=2), 260),
+    ("mxfp4_gemm_shared", mi.GPTOSS.replace(d_model=512, d_ff=1024, n_experts=6, top_k=2, n_shared=1), 200),
+    ("nvfp4_gemm_shared_zipf", mi.BANK.replace(d_model=768, d_ff=512, n_experts=10, top_k=3, n_shared=2), 230),
 ]
 
 
@@ -395,6 +397,50 @@ def test_q4_gemm_is_default_for_prefill_sized_groups():
         moe.moe_profile_enable(False)
         assert want in prof, (T, sorted(prof))
         H.full_check(hl, res)
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "int4"])
+def test_q4_gemm_through_a_slot_map(fmt, monkeypatch):
+    """The 4-bit tensor-core path addressing experts through a slot map (the
+    expert cache's placement): experts stored in a permuted order give
+    bit-identical outputs to the identity placement; an expert marked
+    non-resident (-1) is skipped and its rows are left as they were."""
+    import expert_ffn_layer_route_b200 as moe
+    monkeypatch.setenv("MOE_FFN_PATH", "gemm")
+    shape = mi.BANK.replace(d_model=1024, d_ff=1024, n_experts=6, top_k=2, wdtype=fmt, zipf_s=0.0)
+    T = 160
+    hl, dl = _layer(shape, T, 35)
+    ref = H.run_steps(dl)
+    perm = torch.tensor([3, 0, 5, 1, 4, 2], dtype=torch.int32)  # logical e -> physical slot perm[e]
+    phys = {}
+    for key, v in dl["experts"].items():
+        if key in ("g13", "g2"):
+            phys[key] = v  # global scales are indexed by the logical expert
+            continue
+        t = torch.empty_like(v)
+        t[perm.long().cuda()] = v
+        phys[key] = t
+    desc = moe.make_desc(shape, T)
+    ws = torch.empty(moe.moe_workspace_size(desc), dtype=torch.uint8, device="cuda")
+    for missing in (None, 4):
+        smap = perm.clone()
+        if missing is not None:
+            smap[missing] = -1
+        smap_d = smap.cuda()  # kept alive until the kernel has run
+        w = moe.make_weights(phys, slot_map=smap_d, n_physical=6)
+        y = torch.full_like(ref["y"], 3.0)
+        moe.moe_grouped_ffn(desc, w, None, ref["offsets"], ref["row_token"], dl["x"], y, None, ws)
+        torch.cuda.synchronize()
+        assert moe.moe_get_last_error() == 0
+        if missing is None:
+            assert torch.equal(y, ref["y"])
+        else:
+            offs = ref["offsets"].cpu().tolist()
+            lo, hi = offs[missing], offs[missing + 1]
+            keep = torch.ones(y.shape[0], dtype=torch.bool)
+            keep[lo:hi] = False
+            assert torch.equal(y[keep.cuda()], ref["y"][keep.cuda()])
+            assert bool((y[lo:hi] == 3.0).all())
 
 
 def test_q4_gemm_full_size_mixtral_mxfp4_prefill_sampled():
