@@ -144,7 +144,7 @@ __device__ __forceinline__ Item decode_item(const FfnArgs& a, int item, int ntil
   return it;
 }
 
-template <int F, int NG, bool kGateUp, int MINB, bool kHalf>
+template <int F, int NG, bool kGateUp, int MINB, bool kHalf, bool kSplit>
 __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid_constant__ FfnArgs a) {
   using Tr = FmtTraits<F>;
   constexpr int KC = Tr::kc;
@@ -248,6 +248,12 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
   tc::fence_after_sync();
   const int ngroups = *s_ngroups;
   const int n_items = s_gitem[ngroups];
+  // split K (one column group only): item i of the launch is slice i % S of
+  // item i / S; every block sees the same n_items, so a launch whose items
+  // would overflow the partial buffers runs unsplit everywhere
+  int S = (kSplit && NG == 1) ? a.split : 1;
+  if (S > 1 && (int64_t)n_items * S > a.split_cap) S = 1;
+  const int n_work = n_items * S;
   const int K = a.K;
   const int srow = Tr::blk ? (K / Tr::blk) * Tr::sbytes : 0;
   const int nchunks = ceil_div(K, KC);
@@ -264,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
   // block b takes items b, b + gridDim.x, ... and consumers follow the same
   // sequence on their own (the claims cost more than the balance gained:
   // gpt-oss stage 2 at T=64, 2.97 items per block, 114 vs 108 us).
-  const bool dynamic = n_items > 3 * (int)gridDim.x;
+  const bool dynamic = n_work > 3 * (int)gridDim.x;
 
   if (warp == kConsumerWarps) {
     // ===================================================== producer warp
@@ -276,12 +282,14 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
       const uint64_t pol_x = l2_evict_last_policy();
       uint32_t cnt = 0;
       int item = blockIdx.x;
-      // claim a ring's depth (+1) ahead of the item's end: the answer is back
-      // before the producer needs it, and the claimed item waits only that long
-      const int claim_at = max(0, nchunks - 1 - nstage);
-      while (item < n_items && !*s_abort) {
-        int next_item = n_items;
-        const Item it = decode_item<F>(a, item, ntile, s_gitem, s_gexp, ngroups, s_offs);
+      while (item < n_work && !*s_abort) {
+        int next_item = n_work;
+        const int base = item / S, slice = item - base * S;
+        const int ch_lo = slice * nchunks / S, ch_hi = (slice + 1) * nchunks / S;
+        // claim a ring's depth (+1) ahead of the item's end: the answer is back
+        // before the producer needs it, and the claimed item waits only that long
+        const int claim_at = max(ch_lo, ch_hi - 1 - nstage);
+        const Item it = decode_item<F>(a, base, ntile, s_gitem, s_gexp, ngroups, s_offs);
         const int r0 = it.tile * rows_per_item;
         const int nrows = min(rows_per_item, a.N - r0);
         const CUtensorMap* tw = it.shared_idx >= 0 ? &a.tm_wsh : &a.tm_w;
@@ -314,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
         const int nbox_w = kGateUp ? 2 : (!kHalf && nrows > kBoxRows ? 2 : 1);
         constexpr int kBoxH = kGateUp ? kItemRows : kBoxRows;  // rows per weight box
         const int c0 = it.pass * XCOLS;
-        for (int ch = 0; ch < nchunks && !*s_abort; ++ch) {
+        for (int ch = ch_lo; ch < ch_hi && !*s_abort; ++ch) {
           if (ch == claim_at) next_item = dynamic ? (int)gridDim.x + atomicAdd(a.work_ctr, 1) : item + (int)gridDim.x;
           const int s = cnt % nstage;
           if (!mbar_wait(&empty[s], ((cnt / nstage) & 1u) ^ 1u)) {
@@ -407,10 +415,12 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
       }
       item = s_hdr[s];
       if (item < 0) break;
-    } else if (item >= n_items) {
+    } else if (item >= n_work) {
       break;
     }
-    const Item it = decode_item<F>(a, item, ntile, s_gitem, s_gexp, ngroups, s_offs);
+    const int base = item / S, slice = item - base * S;
+    const int ch_lo = slice * nchunks / S, ch_hi = (slice + 1) * nchunks / S;
+    const Item it = decode_item<F>(a, base, ntile, s_gitem, s_gexp, ngroups, s_offs);
     const int r0 = it.tile * rows_per_item;
     const int nrows = min(rows_per_item, a.N - r0);
     const bool active = it.valid && m0 < nrows;
@@ -459,7 +469,18 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
     float tmp[NG][kMT][4];  // INT4 group partials
     float gbias[NG][2];   // INT4 constant part of the group's partials, per column
     const int n_grp = K / 128;
-    for (int ch = 0; ch < nchunks; ++ch) {
+    // INT4: where this lane's columns' constant parts start (row * n_grp), once per item
+    [[maybe_unused]] int gb_off[NG][2];
+    if constexpr (F == kINT4) {
+#pragma unroll
+      for (int q = 0; q < NG; ++q)
+#pragma unroll
+        for (int hc = 0; hc < 2; ++hc) {
+          const int col = c0 + q * 8 + sigma8(2 * c + hc);
+          gb_off[q][hc] = (it.xrow0 + (col < it.n_cols ? col : 0)) * n_grp;
+        }
+    }
+    for (int ch = ch_lo; ch < ch_hi; ++ch) {
       const int s = cnt % nstage;
       const bool work = active && ncols > 0;
       // this chunk's scales of the owned row (issued before the wait for the stage)
@@ -555,11 +576,7 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
               for (int q = 0; q < NQ; ++q) {
                 if (kGuard && q >= ng_act) break;
 #pragma unroll
-                for (int hc = 0; hc < 2; ++hc) {
-                  const int col = c0 + q * 8 + sigma8(2 * c + hc);
-                  const int row = it.xrow0 + (col < it.n_cols ? col : 0);
-                  gbias[q][hc] = __ldg(a.xbias + (int64_t)row * n_grp + grp);
-                }
+                for (int hc = 0; hc < 2; ++hc) gbias[q][hc] = __ldg(a.xbias + gb_off[q][hc] + grp);
               }
             }
           }
@@ -641,6 +658,41 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
       ++cnt;
     }
     if (*s_abort) break;
+    // ------------------------------------------------- split K: slice sums
+    if constexpr (kSplit && NG == 1) {
+      if (S > 1) {
+        if (!(active && ncols > 0)) continue;
+        constexpr int kPartF = kMT * 4;  // this thread's accumulators
+        const size_t thr = (size_t)(warp * 32 + lane) * 8;
+        float* part0 = a.split_part + (size_t)base * S * (kConsumerWarps * 32 * 8) + thr;
+        float* mine = part0 + (size_t)slice * (kConsumerWarps * 32 * 8);
+#pragma unroll
+        for (int mt = 0; mt < kMT; ++mt)
+          __stcg(reinterpret_cast<float4*>(mine) + mt, make_float4(acc[0][mt][0], acc[0][mt][1], acc[0][mt][2], acc[0][mt][3]));
+        __threadfence();
+        __syncwarp();
+        int old = 0;
+        if (lane == 0) old = atomicAdd(a.split_ctr + (size_t)base * kConsumerWarps + warp, 1);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        if (old != S - 1) continue;  // another slice's warp finishes these rows
+        __threadfence();
+        // every slice's partial, summed in slice order (the same sum whichever warp is last)
+#pragma unroll
+        for (int mt = 0; mt < kMT; ++mt) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(part0) + mt);
+          acc[0][mt][0] = v.x; acc[0][mt][1] = v.y; acc[0][mt][2] = v.z; acc[0][mt][3] = v.w;
+        }
+        for (int sl = 1; sl < S; ++sl) {
+          const float4* ps = reinterpret_cast<const float4*>(part0 + (size_t)sl * (kConsumerWarps * 32 * 8));
+#pragma unroll
+          for (int mt = 0; mt < kMT; ++mt) {
+            const float4 v = __ldcg(ps + mt);
+            acc[0][mt][0] += v.x; acc[0][mt][1] += v.y; acc[0][mt][2] += v.z; acc[0][mt][3] += v.w;
+          }
+        }
+        static_assert(kPartF <= 8, "partial slots per thread");
+      }
+    }
     // ---------------------------------------------------------- epilogue
     if (active && ncols > 0) {
 #pragma unroll
@@ -699,11 +751,11 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
 }
 
 // ------------------------------------------------------------------ host side
-template <int F, int NG, bool GU, int MINB, bool HALF>
+template <int F, int NG, bool GU, int MINB, bool HALF, bool SPLIT = false>
 static cudaError_t launch_one(const FfnArgs& a, int grid, size_t smem, cudaStream_t st) {
-  auto kern = ffn_stream_kernel<F, NG, GU, MINB, HALF>;
+  auto kern = ffn_stream_kernel<F, NG, GU, MINB, HALF, SPLIT>;
   {
-    cudaError_t err = set_dyn_smem_once<ffn_stream_kernel<F, NG, GU, MINB, HALF>>(smem);
+    cudaError_t err = set_dyn_smem_once<ffn_stream_kernel<F, NG, GU, MINB, HALF, SPLIT>>(smem);
     if (err != cudaSuccess) return err;
   }
   if (a.tmem_alloc > 0) {
@@ -721,6 +773,15 @@ static cudaError_t launch_one(const FfnArgs& a, int grid, size_t smem, cudaStrea
 template <int F, bool GU>
 static cudaError_t dispatch_ng(const FfnArgs& a, int ng, int minb, bool half, int grid, size_t smem,
                                cudaStream_t st) {
+  if (a.split > 1) {  // split K: one column group
+    if (half) {
+      if (minb == 3) return launch_one<F, 1, GU, 3, true, true>(a, grid, smem, st);
+      return launch_one<F, 1, GU, 2, true, true>(a, grid, smem, st);
+    }
+    if (minb == 3) return launch_one<F, 1, GU, 3, false, true>(a, grid, smem, st);
+    if (minb == 2) return launch_one<F, 1, GU, 2, false, true>(a, grid, smem, st);
+    return launch_one<F, 1, GU, 1, false, true>(a, grid, smem, st);
+  }
   if (half) {  // one column group, two or three blocks per SM
     if (minb == 3) return launch_one<F, 1, GU, 3, true>(a, grid, smem, st);
     return launch_one<F, 1, GU, 2, true>(a, grid, smem, st);
@@ -910,7 +971,27 @@ cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers&
   const int ntile = ceil_div(a.N, rows_per_item);
   const long max_items = (long)(a.n_shared + (a.E < T * a.k ? a.E : T * a.k)) * ntile;
   const long slots = (long)n_sms * minb;
-  int grid = (int)(max_items < slots ? max_items : slots);
+  // Split K (off by default; MOE_FFN_SPLIT=S asks for S slices): each block
+  // decodes a slice of an item's K chunks, for batches of a few tokens whose
+  // items would leave most block slots idle; one pass per item (T <= 8)
+  // keeps the item count the bound computed here.  Measured on B200 it does
+  // not pay: the gpt-oss-shaped layer at T = 1 with 4 slices takes 54.8 vs
+  // 53.5 us per layer, because a block's time there is set by the launch
+  // ramp, its setup, the first burst of loads all blocks issue at once and
+  // the epilogue, not by its decode work (timestamps per block: stage 1 takes
+  // ~16 us after its predecessor ends either way), and every slice re-reads
+  // the item's block scales.
+  int split = 1;
+  if (ng == 1 && a.split_cap > 0 && T <= 8 && max_items > 0) {
+    const int nch = ceil_div(a.K, fmt_kc(F));
+    if (const char* e = getenv("MOE_FFN_SPLIT")) {
+      const int v = atoi(e);
+      if (v >= 1 && v <= 8 && max_items * v <= a.split_cap && nch >= v) split = v;
+    }
+  }
+  a.split = split;
+  const long work = max_items * split;
+  int grid = (int)(work < slots ? work : slots);
   if (grid < 1) return cudaSuccess;
   switch (F) {
     case kBF16: return gate_up ? dispatch_ng<kBF16, true>(a, ng, minb, half, grid, smem, st) : dispatch_ng<kBF16, false>(a, ng, minb, half, grid, smem, st);

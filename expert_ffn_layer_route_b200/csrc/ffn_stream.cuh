@@ -42,7 +42,20 @@ struct alignas(64) FfnArgs {
   int tmem_alloc;  // TMEM columns allocated per block (power of two >= 32)
   int w_l2_first;        // 1: weight boxes marked evict-first in L2; 0 (default): normal priority
   int32_t* work_ctr;     // launch-wide item counter, zero before the launch
+  // Split K: each item's K chunks in `split` consecutive slices, one work
+  // item each; every consumer warp stores its fp32 partial accumulators, and
+  // the warp that arrives last (per-item, per-warp counters, zero before the
+  // launch) sums the slices in slice order and runs the epilogue.
+  int split;             // slices per item (1: no split; set by the launcher)
+  int split_cap;         // work items the buffers below hold (0: split off)
+  int32_t* split_ctr;    // [split_cap][consumer warps] arrivals
+  float* split_part;     // [split_cap][consumer threads][8] fp32 partials
 };
+
+// Capacity of the split-K buffers (work items), and their sizes in bytes.
+constexpr int kStreamSplitCap = 512;
+constexpr int kStreamSplitCtrInts = kStreamSplitCap * 8;
+constexpr size_t kStreamSplitPartBytes = (size_t)kStreamSplitCap * 256 * 8 * sizeof(float);
 
 // Launch one stage (gate_up: stage 1 with SwiGLU; else stage 2) of the
 // streaming FFN.  The caller fills everything but the tensor maps, which are

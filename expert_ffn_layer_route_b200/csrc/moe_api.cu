@@ -30,6 +30,11 @@ cudaError_t launch_prep_rows(const void* src, int rows, int K, int mode, void* d
                              cudaStream_t st);
 cudaError_t launch_combine(const void* y, const int32_t* inv, const float* gw, const void* y_shared, int n_shared,
                            int T, int d, int k, void* out, cudaStream_t st);
+bool route_prep_small_supported(const moe_layer_desc& d);
+cudaError_t launch_route_prep_small(const moe_layer_desc& dsc, const void* x, const void* wr, const float* bias,
+                                    int32_t* topk_idx, float* topk_w, int32_t* offsets, int32_t* row_token,
+                                    int32_t* inv, int mode, void* xperm, int32_t* xexp, float* gbias, int32_t* zero,
+                                    int n_zero, cudaStream_t st);
 
 }  // namespace moe
 
@@ -60,8 +65,23 @@ int64_t scale_bytes(int f, int64_t N, int64_t K) {
 }
 
 struct Layout {
-  size_t logits, topk_idx, topk_w, offsets, row_token, inv, xperm, xexp, gbias, h, hq, hexp, y, ysh, ctr, total;
+  size_t logits, topk_idx, topk_w, offsets, row_token, inv, xperm, xexp, gbias, h, hq, hexp, y, ysh, ctr, split_part,
+      total;
+  int n_ctr;  // int32 counters at ctr, zeroed by the activation-prep kernel of every call
 };
+
+// Batches of at most this many tokens may split the streaming FFN's items
+// along K (MOE_FFN_SPLIT=S, off by default); their workspace holds the split
+// counters and partial sums.
+constexpr int kSplitMaxT = 8;
+
+// Counters the activation-prep kernel zeroes: the two work counters, plus the
+// split-K arrival counters when a split is asked for.
+int counters_to_zero(const Layout& L) {
+  if (L.n_ctr <= 2) return 2;
+  const char* e = std::getenv("MOE_FFN_SPLIT");
+  return (e && std::atoi(e) > 1) ? L.n_ctr : 2;
+}
 
 Layout layout_of(const moe_layer_desc& d) {
   Layout L{};
@@ -89,7 +109,12 @@ Layout layout_of(const moe_layer_desc& d) {
   L.hexp = take(q ? RT * 4 : 0);
   L.y = take(R * D * 2);
   L.ysh = take(S * T * D * 2);
-  L.ctr = take(2 * 4);  // work counters of the two streaming FFN stages
+  // work counters of the two streaming FFN stages, then (small batches) each
+  // stage's split-K arrival counters
+  const bool split = d.T <= kSplitMaxT;
+  L.n_ctr = 2 + (split ? 2 * kStreamSplitCtrInts : 0);
+  L.ctr = take((size_t)L.n_ctr * 4);
+  L.split_part = take(split ? kStreamSplitPartBytes : 0);  // shared by both stages (they run in turn)
   L.total = o;
   return L;
 }
@@ -145,9 +170,45 @@ moe_status check_weights(const moe_layer_desc& d, const moe_weights* w, int n_ex
   return MOE_OK;
 }
 
+// Which FFN path a call takes, and the activation-row format that path reads.
+struct FfnPlan {
+  bool use_gemm;     // tensor-core grouped GEMM (else the weight-streaming kernel)
+  bool q_bf16_acts;  // 4-bit on the GEMM path with bf16 activation rows (MXFP4)
+  bool int4_stream;  // INT4 on the streaming path (offset decode: reordered rows + group constants)
+  int mode;          // activation prep: 0 fp16 scaled, 1 fp16 scaled for the INT4 decode, 2 bf16 copy
+};
+
+FfnPlan ffn_plan(const moe_layer_desc& d) {
+  const int f = d.wdtype;
+  const bool q = is4bit(f);
+  const int F = d.d_ff, D = d.d_model;
+  // Path: the tcgen05 grouped GEMM when experts average at least 64 rows
+  // (prefill-sized groups; bf16 weights, or 4-bit weights decoded to 16-bit
+  // tiles in shared memory), else the weight-streaming kernel.
+  // MOE_FFN_PATH=stream|gemm overrides the choice where both can run.
+  const bool gemm_ok = q ? (gemm_q4_supported(f, F, D, true) && gemm_q4_supported(f, D, F, false))
+                         : (gemm_path_supported(f, F, D, true) && gemm_path_supported(f, D, F, false));
+  FfnPlan p{};
+  p.use_gemm = gemm_ok && (int64_t)d.T * d.top_k >= 64LL * d.n_experts;
+  if (const char* e = getenv("MOE_FFN_PATH")) {
+    if (!strcmp(e, "stream")) p.use_gemm = false;
+    if (!strcmp(e, "gemm")) p.use_gemm = gemm_ok;
+  }
+  // Activation rows: bf16 copies (bf16 weights; MXFP4 on the tensor-core
+  // path), fp16 scaled by a power of two per row (the 4-bit formats
+  // otherwise), for the streaming INT4 decode also reordered with the
+  // per-group constants.
+  p.q_bf16_acts = q && p.use_gemm && gemm_q4_bf16_activations(f);
+  p.int4_stream = f == MOE_W_INT4_G128 && !p.use_gemm;
+  p.mode = (!q || p.q_bf16_acts) ? 2 : (p.int4_stream ? 1 : 0);
+  return p;
+}
+
+// x_prepped: the activation rows (and the stage counters) were already
+// written by the fused small-batch routing kernel.
 moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, const moe_weights* shared,
                             const int32_t* offsets, const int32_t* row_token, const void* x, void* y_perm,
-                            void* y_shared, uint8_t* ws, cudaStream_t st) {
+                            void* y_shared, uint8_t* ws, cudaStream_t st, bool x_prepped = false) {
   const Layout L = layout_of(d);
   const int f = d.wdtype;
   const bool q = is4bit(f);
@@ -160,30 +221,17 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
   __half* hq = reinterpret_cast<__half*>(ws + L.hq);
   int32_t* hexp = reinterpret_cast<int32_t*>(ws + L.hexp);
-  // Path: the tcgen05 grouped GEMM when experts average at least 64 rows
-  // (prefill-sized groups; bf16 weights, or 4-bit weights decoded to 16-bit
-  // tiles in shared memory), else the weight-streaming kernel.
-  // MOE_FFN_PATH=stream|gemm overrides the choice where both can run.
-  const bool gemm_ok = q ? (gemm_q4_supported(f, F, D, true) && gemm_q4_supported(f, D, F, false))
-                         : (gemm_path_supported(f, F, D, true) && gemm_path_supported(f, D, F, false));
-  bool use_gemm = gemm_ok && (int64_t)T * k >= 64LL * E;
-  if (const char* e = getenv("MOE_FFN_PATH")) {
-    if (!strcmp(e, "stream")) use_gemm = false;
-    if (!strcmp(e, "gemm")) use_gemm = gemm_ok;
-  }
-  // Activation rows: bf16 copies (bf16 weights; MXFP4 on the tensor-core
-  // path), fp16 scaled by a power of two per row (the 4-bit formats
-  // otherwise), for the streaming INT4 decode also reordered with the
-  // per-group constants.
-  const bool q_bf16_acts = q && use_gemm && gemm_q4_bf16_activations(f);
-  const bool int4_stream = f == MOE_W_INT4_G128 && !use_gemm;
-  float* gbias = int4_stream ? reinterpret_cast<float*>(ws + L.gbias) : nullptr;
-  const int mode = (!q || q_bf16_acts) ? 2 : (int4_stream ? 1 : 0);
+  const FfnPlan plan = ffn_plan(d);
+  const bool use_gemm = plan.use_gemm, q_bf16_acts = plan.q_bf16_acts;
+  float* gbias = plan.int4_stream ? reinterpret_cast<float*>(ws + L.gbias) : nullptr;
+  const int mode = plan.mode;
   // activation rows in expert order (routed rows, then every token once per shared expert)
   // (also zeroes the work counters of both FFN stages)
   int32_t* ctr = reinterpret_cast<int32_t*>(ws + L.ctr);
-  err = launch_prep_rows(x, RT, D, mode, xperm, xexp, gbias, row_token, R, T, ctr, 2, st);
-  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  if (!x_prepped) {
+    err = launch_prep_rows(x, RT, D, mode, xperm, xexp, gbias, row_token, R, T, ctr, counters_to_zero(L), st);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+  }
   auto fill = [&](FfnArgs& a, FfnPointers& p, bool stage1) {
     std::memset(&a, 0, sizeof(a));
     std::memset(&p, 0, sizeof(p));
@@ -270,6 +318,12 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
   a1.xexp = q ? xexp : nullptr;
   a1.xbias = gbias;
   a1.work_ctr = ctr;
+  const bool split_buffers = counters_to_zero(L) > 2;
+  if (split_buffers) {
+    a1.split_cap = kStreamSplitCap;
+    a1.split_ctr = ctr + 2;
+    a1.split_part = reinterpret_cast<float*>(ws + L.split_part);
+  }
   a1.out_routed = h;
   a1.out_shared = nullptr;
   int unsup = 0;
@@ -295,6 +349,11 @@ moe_status grouped_ffn_impl(const moe_layer_desc& d, const moe_weights* routed, 
   a2.xexp = h_f16 ? hexp : nullptr;
   a2.xbias = gbias;
   a2.work_ctr = ctr + 1;
+  if (split_buffers) {
+    a2.split_cap = kStreamSplitCap;
+    a2.split_ctr = ctr + 2 + kStreamSplitCtrInts;
+    a2.split_part = reinterpret_cast<float*>(ws + L.split_part);
+  }
   a2.out_routed = static_cast<__nv_bfloat16*>(y_perm);
   a2.out_shared = static_cast<__nv_bfloat16*>(y_shared);
   if (use_gemm && q)
@@ -412,14 +471,25 @@ moe_status moe_layer_forward(const moe_layer_desc* desc, const void* x, const vo
   int32_t* offs = reinterpret_cast<int32_t*>(ws + L.offsets);
   int32_t* rtok = reinterpret_cast<int32_t*>(ws + L.row_token);
   int32_t* inv = reinterpret_cast<int32_t*>(ws + L.inv);
-  cudaError_t err = launch_route_topk(*desc, x, w_router, logit_bias, reinterpret_cast<float*>(ws + L.logits), idx,
-                                      gw, st);
-  if (err != cudaSuccess) return MOE_ERR_CUDA;
-  err = launch_permute(idx, desc->T, desc->top_k, desc->n_experts, offs, rtok, inv, st);
-  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  const bool fused = route_prep_small_supported(*desc);
+  cudaError_t err;
+  if (fused) {
+    // small batch: router, top-k, permutation and activation rows in one launch
+    const FfnPlan plan = ffn_plan(*desc);
+    err = launch_route_prep_small(*desc, x, w_router, logit_bias, idx, gw, offs, rtok, inv, plan.mode, ws + L.xperm,
+                                  reinterpret_cast<int32_t*>(ws + L.xexp),
+                                  plan.int4_stream ? reinterpret_cast<float*>(ws + L.gbias) : nullptr,
+                                  reinterpret_cast<int32_t*>(ws + L.ctr), counters_to_zero(L), st);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+  } else {
+    err = launch_route_topk(*desc, x, w_router, logit_bias, reinterpret_cast<float*>(ws + L.logits), idx, gw, st);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+    err = launch_permute(idx, desc->T, desc->top_k, desc->n_experts, offs, rtok, inv, st);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+  }
   void* y = ws + L.y;
   void* ysh = desc->n_shared ? ws + L.ysh : nullptr;
-  s = grouped_ffn_impl(*desc, routed, shared, offs, rtok, x, y, ysh, ws, st);
+  s = grouped_ffn_impl(*desc, routed, shared, offs, rtok, x, y, ysh, ws, st, fused);
   if (s != MOE_OK) return s;
   return from_cuda(launch_combine(y, inv, gw, ysh, desc->n_shared, desc->T, desc->d_model, desc->top_k, out, st));
 }

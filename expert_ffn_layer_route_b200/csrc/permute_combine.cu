@@ -18,6 +18,7 @@
 #include "common.cuh"
 #include "launch.cuh"
 #include "profile.cuh"
+#include "route_device.cuh"
 
 namespace moe {
 
@@ -137,14 +138,13 @@ static int row_threads(int K) {
   int t = ((K / 8 + 31) / 32) * 32;
   return t < kRowThreadsMin ? kRowThreadsMin : (t > kRowThreadsMax ? kRowThreadsMax : t);
 }
-enum PrepMode : int { kF16 = 0, kF16Int4 = 1, kCopyBf16 = 2 };
-
 template <int kMode>
 __global__ void __launch_bounds__(kRowThreadsMax)
     prep_rows_kernel(const __nv_bfloat16* __restrict__ src, int K, void* __restrict__ dst,
                      int32_t* __restrict__ rexp, float* __restrict__ gbias, const int32_t* __restrict__ gather,
                      int n_gather, int n_tok, int32_t* __restrict__ zero, int n_zero) {
   pdl_wait_and_trigger();
+  __shared__ float red[kRowThreadsMax / 32];
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
   const int nth = blockDim.x;
@@ -154,79 +154,11 @@ __global__ void __launch_bounds__(kRowThreadsMax)
   // a gathered row past the grouped rows (a pair the permutation dropped)
   // has no source: it is written as zeros
   const bool have = !gather || (unsigned)srow < (unsigned)n_tok;
-  const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)(have ? srow : 0) * K);
-  const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-  const int nchunk = K / 8;
-  if constexpr (kMode == kCopyBf16) {
-    uint4* d = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + (size_t)row * K);
-    for (int c = tid; c < nchunk; c += nth) d[c] = have ? __ldg(s + c) : z4;
-    return;
-  }
-  float amax = 0.f;
-  for (int c = tid; c < nchunk; c += nth) {
-    const uint4 u = have ? __ldg(s + c) : z4;
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      amax = fmaxf(amax, fabsf(bf16_bits_to_f32(w[q] & 0xffffu)));
-      amax = fmaxf(amax, fabsf(bf16_bits_to_f32(w[q] >> 16)));
-    }
-  }
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  __shared__ float red[kRowThreadsMax / 32];
-  if ((tid & 31) == 0) red[tid >> 5] = amax;
-  __syncthreads();
-  amax = red[0];
-#pragma unroll
-  for (int w = 1; w < nth / 32; ++w) amax = fmaxf(amax, red[w]);
-  int p = 0;
-  if (amax > 0.f && amax <= 3.0e38f) {
-    int ex;
-    frexpf(amax, &ex);  // amax = m * 2^ex, m in [0.5, 1)
-    p = ex - 15;        // floor(log2(amax)) - 14
-  }
-  if (tid == 0) rexp[row] = p;
-  const float scale = ldexpf(1.f, -p);
-  uint4* d = reinterpret_cast<uint4*>(static_cast<__half*>(dst) + (size_t)row * K);
-  // every thread runs the same number of rounds so that the 16-lane group
-  // sums below see full warps (nchunk is a multiple of 16 for INT4)
-  for (int base = 0; base < nchunk; base += nth) {
-    const int c = base + tid;
-    const bool on = c < nchunk;
-    float f[8];
-    if (on) {
-      const uint4 u = have ? __ldg(s + c) : z4;
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        f[2 * q] = bf16_bits_to_f32(w[q] & 0xffffu) * scale;
-        f[2 * q + 1] = bf16_bits_to_f32(w[q] >> 16) * scale;
-      }
-    } else {
-#pragma unroll
-      for (int q = 0; q < 8; ++q) f[q] = 0.f;
-    }
-    __half h[8];
-    if constexpr (kMode == kF16Int4) {
-      const int order[8] = {0, 4, 1, 5, 2, 6, 3, 7};
-      double even = 0.0, odd = 0.0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int k = order[q];
-        h[q] = __float2half_rn((k & 1) ? f[k] * 0.0625f : f[k]);
-        if (k & 1) odd += (double)__half2float(h[q]); else even += (double)__half2float(h[q]);
-      }
-      double part = 1032.0 * even + 1152.0 * odd;
-#pragma unroll
-      for (int off = 8; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-      if (on && (tid & 15) == 0) gbias[(size_t)row * (K / 128) + (c >> 4)] = (float)part;
-    } else {
-#pragma unroll
-      for (int q = 0; q < 8; ++q) h[q] = __float2half_rn(f[q]);
-    }
-    if (on) d[c] = *reinterpret_cast<uint4*>(h);
-  }
+  const __nv_bfloat16* s = have ? src + (size_t)srow * K : nullptr;
+  const size_t esz = kMode == kCopyBf16 ? sizeof(__nv_bfloat16) : sizeof(__half);
+  void* d = static_cast<uint8_t*>(dst) + (size_t)row * K * esz;
+  prep_row<kMode>(s, K, d, rexp ? rexp + row : nullptr, gbias ? gbias + (size_t)row * (K / 128) : nullptr, tid, nth,
+                  red);
 }
 
 // mode: 0 fp16 scaled, 1 fp16 scaled for the INT4 decode (+ gbias), 2 bf16 copy.

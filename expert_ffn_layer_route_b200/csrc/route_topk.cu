@@ -23,99 +23,31 @@
 #include "common.cuh"
 #include "launch.cuh"
 #include "profile.cuh"
+#include "route_device.cuh"
 
 namespace moe {
-
-constexpr int kRouterExperts = 4;  // experts per block
-constexpr int kRouterThreads = 256;
 
 template <bool kFp32Router, int kRouterTokens>
 __global__ void __launch_bounds__(kRouterThreads)
     router_logits_kernel(const __nv_bfloat16* __restrict__ x, const void* __restrict__ wr,
                          const float* __restrict__ bias, float* __restrict__ logits, int T, int d, int E) {
+  // the router weights are not written by a kernel this one may overlap: the
+  // first token tile brings its experts' rows into L2 before the wait
+  if (blockIdx.x == 0) {
+    const size_t esz = kFp32Router ? 4 : 2;
+    const int e_lo = blockIdx.y * kRouterExperts;
+    const size_t nbytes = (size_t)(min(E, e_lo + kRouterExperts) - e_lo) * d * esz;
+    const char* w0 = static_cast<const char*>(wr) + (size_t)e_lo * d * esz;
+    for (size_t o = (size_t)threadIdx.x * 128; o < nbytes; o += (size_t)kRouterThreads * 128)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(w0 + o));
+  }
   pdl_wait_and_trigger();
+  __shared__ float part[(kRouterThreads / 32) * kRouterTokens * kRouterExperts];
   const int t0 = blockIdx.x * kRouterTokens;
   const int e0 = blockIdx.y * kRouterExperts;
-  const int tid = threadIdx.x;
-  const int nt = min(kRouterTokens, T - t0);
-  const int ne = min(kRouterExperts, E - e0);
-  float acc[kRouterTokens][kRouterExperts];
-#pragma unroll
-  for (int a = 0; a < kRouterTokens; ++a)
-#pragma unroll
-    for (int b = 0; b < kRouterExperts; ++b) acc[a][b] = 0.f;
-
-  const int nchunk = d / 8;
-  for (int c = tid; c < nchunk; c += kRouterThreads) {
-    float wv[kRouterExperts][8];
-#pragma unroll
-    for (int b = 0; b < kRouterExperts; ++b) {
-      const int e = e0 + (b < ne ? b : 0);
-      if constexpr (kFp32Router) {
-        const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(wr) + (size_t)e * d + c * 8);
-        float4 u0 = __ldg(p), u1 = __ldg(p + 1);
-        wv[b][0] = u0.x; wv[b][1] = u0.y; wv[b][2] = u0.z; wv[b][3] = u0.w;
-        wv[b][4] = u1.x; wv[b][5] = u1.y; wv[b][6] = u1.z; wv[b][7] = u1.w;
-      } else {
-        uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(wr) + (size_t)e * d + c * 8));
-        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          wv[b][2 * q] = bf16_bits_to_f32(w4[q] & 0xffffu);
-          wv[b][2 * q + 1] = bf16_bits_to_f32(w4[q] >> 16);
-        }
-      }
-    }
-#pragma unroll
-    for (int a = 0; a < kRouterTokens; ++a) {
-      const int t = t0 + (a < nt ? a : 0);
-      uint4 u = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d + c * 8));
-      const uint32_t x4[4] = {u.x, u.y, u.z, u.w};
-      float xv[8];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        xv[2 * q] = bf16_bits_to_f32(x4[q] & 0xffffu);
-        xv[2 * q + 1] = bf16_bits_to_f32(x4[q] >> 16);
-      }
-#pragma unroll
-      for (int b = 0; b < kRouterExperts; ++b)
-#pragma unroll
-        for (int q = 0; q < 8; ++q) acc[a][b] = __fadd_rn(acc[a][b], __fmul_rn(xv[q], wv[b][q]));
-    }
-  }
-  // warp butterfly (identical association in every lane and every column)
-#pragma unroll
-  for (int a = 0; a < kRouterTokens; ++a)
-#pragma unroll
-    for (int b = 0; b < kRouterExperts; ++b)
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) acc[a][b] = __fadd_rn(acc[a][b], __shfl_xor_sync(0xffffffffu, acc[a][b], off));
-
-  __shared__ float part[kRouterThreads / 32][kRouterTokens * kRouterExperts];
-  const int warp = tid >> 5, lane = tid & 31;
-  if (lane == 0) {
-#pragma unroll
-    for (int a = 0; a < kRouterTokens; ++a)
-#pragma unroll
-      for (int b = 0; b < kRouterExperts; ++b) part[warp][a * kRouterExperts + b] = acc[a][b];
-  }
-  __syncthreads();
-  if (tid < kRouterTokens * kRouterExperts) {
-    const int a = tid / kRouterExperts, b = tid % kRouterExperts;
-    float s = part[0][tid];
-#pragma unroll
-    for (int w = 1; w < kRouterThreads / 32; ++w) s = __fadd_rn(s, part[w][tid]);
-    if (a < nt && b < ne) {
-      const int e = e0 + b;
-      if (bias != nullptr) s = __fadd_rn(s, __ldg(bias + e));
-      logits[(size_t)(t0 + a) * E + e] = s;
-    }
-  }
-}
-
-// (value, index) ordering: larger value first, then lower index.  NaN never wins.
-__device__ __forceinline__ bool beats(float v, int i, float w, int j) {
-  return (v > w) || (v == w && i < j);
+  router_tile<kFp32Router, kRouterTokens>(x, wr, bias, T, d, E, t0, e0, part, [&](int a, int b, float v) {
+    logits[(size_t)(t0 + a) * E + e0 + b] = v;
+  });
 }
 
 __global__ void __launch_bounds__(256)
@@ -123,46 +55,8 @@ __global__ void __launch_bounds__(256)
                 int T, int E, int k) {
   pdl_wait_and_trigger();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
   if (warp >= T) return;
-  const float* lt = logits + (size_t)warp * E;
-  int prev_i = -1;
-  float prev_v = __int_as_float(0x7f800000);  // +inf: everything is below the previous pick
-  float my_v = 0.f;
-  int my_i = -1;
-  for (int j = 0; j < k; ++j) {
-    // best element strictly after (prev_v, prev_i) in the total order
-    float bv = __int_as_float(0xff800000);  // -inf
-    int bi = 0x7fffffff;
-    for (int e = lane; e < E; e += 32) {
-      const float v = lt[e];
-      if (v != v) continue;  // NaN is never selected
-      if (!beats(prev_v, prev_i, v, e)) continue;
-      if (beats(v, e, bv, bi)) { bv = v; bi = e; }
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-      if (beats(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-    }
-    if (bi == 0x7fffffff || bi < 0 || bi >= E) {
-      bi = -1;
-      if (lane == 0) set_status(MOE_ERR_DEVICE_INDEX);
-    }
-    if (lane == j) { my_v = bv; my_i = bi; }
-    prev_v = bv;
-    prev_i = bi;
-  }
-  // gates: softmax over the selected logits (lane j holds pick j; pick 0 is the max)
-  const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
-  const float ex = (lane < k) ? expf(my_v - vmax) : 0.f;
-  float sum = 0.f;
-  for (int j = 0; j < k; ++j) sum = __fadd_rn(sum, __shfl_sync(0xffffffffu, ex, j));
-  if (lane < k) {
-    topk_idx[(size_t)warp * k + lane] = my_i;
-    topk_w[(size_t)warp * k + lane] = ex / sum;
-  }
+  topk_warp(logits + (size_t)warp * E, E, k, topk_idx + (size_t)warp * k, topk_w + (size_t)warp * k);
 }
 
 cudaError_t launch_route_topk(const moe_layer_desc& dsc, const void* x, const void* wr, const float* bias,

@@ -73,6 +73,28 @@ def test_half_items_forced_in_both_stages(half, monkeypatch):
         print(f"half={half} {shape.name} T={T}: rel err {rel:.2e}, ambiguous {n_amb}")
 
 
+@pytest.mark.parametrize("split", ["1", "2", "3", "4"])
+def test_split_k_forced(split, monkeypatch):
+    """The streaming FFN's split-K items (each item's K chunks in S slices,
+    the slice partials summed by the last-arriving warp; by default used when
+    a batch of at most 8 tokens would leave most block slots idle) forced to
+    1-4 slices for every format, against the oracle, and bit-identical on a
+    second run (the slice sums are taken in slice order whichever warp
+    arrives last)."""
+    monkeypatch.setenv("MOE_FFN_SPLIT", split)
+    for shape, T in [(mi.GPTOSS.replace(n_experts=16), 1),
+                     (mi.GPTOSS.replace(n_experts=16), 7),
+                     (mi.KIMI.replace(d_model=2048, d_ff=384, n_experts=48), 2),
+                     (mi.BANK.replace(d_model=1024, d_ff=512, n_experts=32), 4),
+                     (mi.TINY.replace(d_model=512, d_ff=640, n_experts=16, top_k=2), 3)]:
+        hl, dl = _layer(shape, T, 23)
+        a = H.run_layer(dl)
+        rel, n_amb = H.full_check(hl, a)
+        out = a["out"].clone()
+        assert torch.equal(H.run_layer(dl)["out"], out)
+        print(f"split={split} {shape.name} T={T}: rel err {rel:.2e}, ambiguous {n_amb}")
+
+
 @pytest.mark.parametrize("seed", [2])
 def test_tiny_seed2(seed):
     hl, dl = _layer(mi.TINY, 16, seed)
