@@ -339,6 +339,10 @@ def run_ours(args):
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
     shape = mi.CONFIGS[args.workload]
+    if args.experts:
+        # a reduced-expert variant of the layer (same d_model, d_ff, top-k and
+        # format), for profiling captures that must stay a few GB on the device
+        shape = shape.replace(n_experts=max(args.experts, shape.top_k))
     T = args.tokens or DEFAULT_TOKENS[args.workload]
     dlay = mi.draw_layer(shape, T, seed=1000 + rank, device=dev)
     desc = moe.make_desc(shape, T)
@@ -720,6 +724,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--tokens", type=int, default=0, help="tokens per step (default: the workload's)")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="routed experts of a reduced layer variant (default: the workload's); for profiling captures")
     ap.add_argument("--workload", choices=sorted(DEFAULT_TOKENS) + ["verify"], default="gptoss_decode")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")

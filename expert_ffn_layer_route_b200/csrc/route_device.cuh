@@ -37,42 +37,64 @@ __device__ __forceinline__ void router_tile(const __nv_bfloat16* __restrict__ x,
 #pragma unroll
     for (int b = 0; b < kExp; ++b) acc[a][b] = 0.f;
 
+  // Per chunk every accumulator adds its 8 products in q order; the loop
+  // nest around that (which operand is held in registers while the other
+  // streams) changes no sum.  Few experts per tile: the experts' weights are
+  // held and the tokens stream; many (small batches): the tokens are held.
   const int nchunk = d / 8;
-  for (int c = tid; c < nchunk; c += kRouterThreads) {
-    float xv[kTok][8];
-#pragma unroll
-    for (int a = 0; a < kTok; ++a) {
-      const int t = t0 + (a < nt ? a : 0);
-      uint4 u = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d + c * 8));
-      const uint32_t x4[4] = {u.x, u.y, u.z, u.w};
+  auto load_w = [&](int e, int c, float (&wv)[8]) {
+    if constexpr (kFp32Router) {
+      const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(wr) + (size_t)e * d + c * 8);
+      float4 u0 = __ldg(p), u1 = __ldg(p + 1);
+      wv[0] = u0.x; wv[1] = u0.y; wv[2] = u0.z; wv[3] = u0.w;
+      wv[4] = u1.x; wv[5] = u1.y; wv[6] = u1.z; wv[7] = u1.w;
+    } else {
+      uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(wr) + (size_t)e * d + c * 8));
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        xv[a][2 * q] = bf16_bits_to_f32(x4[q] & 0xffffu);
-        xv[a][2 * q + 1] = bf16_bits_to_f32(x4[q] >> 16);
+        wv[2 * q] = bf16_bits_to_f32(w4[q] & 0xffffu);
+        wv[2 * q + 1] = bf16_bits_to_f32(w4[q] >> 16);
       }
     }
+  };
+  auto load_x = [&](int a, int c, float (&xv)[8]) {
+    const int t = t0 + (a < nt ? a : 0);
+    uint4 u = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d + c * 8));
+    const uint32_t x4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int b = 0; b < kExp; ++b) {
-      const int e = e0 + (b < ne ? b : 0);
-      float wv[8];
-      if constexpr (kFp32Router) {
-        const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(wr) + (size_t)e * d + c * 8);
-        float4 u0 = __ldg(p), u1 = __ldg(p + 1);
-        wv[0] = u0.x; wv[1] = u0.y; wv[2] = u0.z; wv[3] = u0.w;
-        wv[4] = u1.x; wv[5] = u1.y; wv[6] = u1.z; wv[7] = u1.w;
-      } else {
-        uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(wr) + (size_t)e * d + c * 8));
-        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+    for (int q = 0; q < 4; ++q) {
+      xv[2 * q] = bf16_bits_to_f32(x4[q] & 0xffffu);
+      xv[2 * q + 1] = bf16_bits_to_f32(x4[q] >> 16);
+    }
+  };
+  for (int c = tid; c < nchunk; c += kRouterThreads) {
+    if constexpr (kExp <= kRouterExperts) {
+      float wv[kExp][8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          wv[2 * q] = bf16_bits_to_f32(w4[q] & 0xffffu);
-          wv[2 * q + 1] = bf16_bits_to_f32(w4[q] >> 16);
-        }
+      for (int b = 0; b < kExp; ++b) load_w(e0 + (b < ne ? b : 0), c, wv[b]);
+#pragma unroll
+      for (int a = 0; a < kTok; ++a) {
+        float xv[8];
+        load_x(a, c, xv);
+#pragma unroll
+        for (int b = 0; b < kExp; ++b)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) acc[a][b] = __fadd_rn(acc[a][b], __fmul_rn(xv[q], wv[b][q]));
       }
+    } else {
+      float xv[kTok][8];
 #pragma unroll
-      for (int a = 0; a < kTok; ++a)
+      for (int a = 0; a < kTok; ++a) load_x(a, c, xv[a]);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) acc[a][b] = __fadd_rn(acc[a][b], __fmul_rn(xv[a][q], wv[q]));
+      for (int b = 0; b < kExp; ++b) {
+        float wv[8];
+        load_w(e0 + (b < ne ? b : 0), c, wv);
+#pragma unroll
+        for (int a = 0; a < kTok; ++a)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) acc[a][b] = __fadd_rn(acc[a][b], __fmul_rn(xv[a][q], wv[q]));
+      }
     }
   }
   // warp butterfly (identical association in every lane and every column)

@@ -31,16 +31,6 @@ template <bool kFp32Router, int kRouterTokens>
 __global__ void __launch_bounds__(kRouterThreads)
     router_logits_kernel(const __nv_bfloat16* __restrict__ x, const void* __restrict__ wr,
                          const float* __restrict__ bias, float* __restrict__ logits, int T, int d, int E) {
-  // the router weights are not written by a kernel this one may overlap: the
-  // first token tile brings its experts' rows into L2 before the wait
-  if (blockIdx.x == 0) {
-    const size_t esz = kFp32Router ? 4 : 2;
-    const int e_lo = blockIdx.y * kRouterExperts;
-    const size_t nbytes = (size_t)(min(E, e_lo + kRouterExperts) - e_lo) * d * esz;
-    const char* w0 = static_cast<const char*>(wr) + (size_t)e_lo * d * esz;
-    for (size_t o = (size_t)threadIdx.x * 128; o < nbytes; o += (size_t)kRouterThreads * 128)
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(w0 + o));
-  }
   pdl_wait_and_trigger();
   __shared__ float part[(kRouterThreads / 32) * kRouterTokens * kRouterExperts];
   const int t0 = blockIdx.x * kRouterTokens;
