@@ -73,6 +73,41 @@ def test_half_items_forced_in_both_stages(half, monkeypatch):
         print(f"half={half} {shape.name} T={T}: rel err {rel:.2e}, ambiguous {n_amb}")
 
 
+FUSED_CASES = [
+    # every token-tile width (1, 2, 4, 8) and activation-row format, fp32 and
+    # bf16 routers, shared experts, 384 experts (a cluster of 16 CTAs where the
+    # device can co-schedule it), 64 (token, slot) pairs, and 7 experts (CTAs
+    # with no router slice)
+    ("mxfp4_T1", mi.GPTOSS.replace(n_experts=16), 1),
+    ("mxfp4_T3", mi.GPTOSS.replace(n_experts=16), 3),
+    ("mxfp4_T8", mi.GPTOSS.replace(n_experts=16), 8),
+    ("int4_shared_T2", mi.KIMI.replace(d_model=896, d_ff=384, n_experts=48), 2),
+    ("int4_shared_T5", mi.KIMI.replace(d_model=896, d_ff=384, n_experts=48), 5),
+    ("int4_E384_T1", mi.KIMI.replace(d_model=1024, d_ff=256, n_experts=384), 1),
+    ("int4_E384_T8_64pairs", mi.KIMI.replace(d_model=1024, d_ff=256, n_experts=384), 8),
+    ("nvfp4_T4", mi.BANK.replace(d_model=1024, d_ff=384, n_experts=32), 4),
+    ("bf16_fp32router_T6", mi.TINY.replace(n_experts=16, top_k=2), 6),
+    ("bf16_E7_T7", mi.TINY.replace(d_model=320, d_ff=96, n_experts=7, top_k=3), 7),
+]
+
+
+@pytest.mark.parametrize("name,shape,T", FUSED_CASES, ids=[c[0] for c in FUSED_CASES])
+def test_fused_small_batch_routing_matches_unfused(name, shape, T, monkeypatch):
+    """The one-launch routing kernel for small batches (router, top-k,
+    permutation, activation rows) forced on and off: the same router tile,
+    top-k and row-prep routines give bit-identical routing, permutation and
+    layer output, and the fused run matches the oracle."""
+    hl, dl = _layer(shape, T, 31)
+    monkeypatch.setenv("MOE_FUSED_ROUTE", "1")
+    a = H.run_layer(dl)
+    rel, n_amb = H.full_check(hl, a)
+    monkeypatch.setenv("MOE_FUSED_ROUTE", "0")
+    b = H.run_layer(dl)
+    for key in ("out", "idx", "gates", "offsets", "row_token", "inv"):
+        assert torch.equal(a[key], b[key]), key
+    print(f"fused {name}: rel err {rel:.2e}, ambiguous {n_amb}")
+
+
 @pytest.mark.parametrize("split", ["1", "2", "3", "4"])
 def test_split_k_forced(split, monkeypatch):
     """The streaming FFN's split-K items (each item's K chunks in S slices,
