@@ -77,6 +77,22 @@ struct FmtTraits<kINT4> {
 
 __device__ __forceinline__ int sigma8(int g) { return (g >> 1) | ((g & 1) << 2); }
 
+// Position in the ring of shared-memory stages: the stage index and the
+// parity of its current fill, advanced without dividing by the run-time ring
+// depth (a division per K chunk costs the consumers' integer pipe ~20
+// instructions twice over).
+struct RingPos {
+  int s;
+  uint32_t ph;
+  int n;
+  __device__ __forceinline__ void next() {
+    if (++s == n) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+};
+
 // Shared-memory header: barriers, flags, offsets [E+1], group table.
 __host__ __device__ constexpr int stream_hdr_bytes(int E, int n_shared) {
   return ((16 * kMaxStages + 64 + 4 * ((E + 4) + 2 * (E + n_shared + 4))) + 1023) & ~1023;
@@ -281,6 +297,7 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
       const uint64_t pol_w = a.w_l2_first ? l2_evict_first_policy() : l2_evict_normal_policy();
       const uint64_t pol_x = l2_evict_last_policy();
       uint32_t cnt = 0;
+      RingPos rp{0, 0u, nstage};
       int item = blockIdx.x;
       while (item < n_work && !*s_abort) {
         int next_item = n_work;
@@ -298,8 +315,8 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
         // gate rows then up rows (stage 1), or kWarpRows rows per warp (stage 2)
         // -- each a contiguous range of the row-major scale matrix.
         for (int j = 0; j < n_sslots && !*s_abort; ++j) {
-          const int s = cnt % nstage;
-          if (!mbar_wait(&empty[s], ((cnt / nstage) & 1u) ^ 1u)) {
+          const int s = rp.s;
+          if (!mbar_wait(&empty[s], rp.ph ^ 1u)) {
             *s_abort = 1;
             break;
           }
@@ -317,6 +334,7 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
                        &full[s]);
           }
           ++cnt;
+          rp.next();
         }
         // boxes of weight rows: stage 1 gate rows r0.. and up rows N+r0..; stage 2 rows r0.., r0+128..
         const int nbox_w = kGateUp ? 2 : (!kHalf && nrows > kBoxRows ? 2 : 1);
@@ -324,8 +342,8 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
         const int c0 = it.pass * XCOLS;
         for (int ch = ch_lo; ch < ch_hi && !*s_abort; ++ch) {
           if (ch == claim_at) next_item = dynamic ? (int)gridDim.x + atomicAdd(a.work_ctr, 1) : item + (int)gridDim.x;
-          const int s = cnt % nstage;
-          if (!mbar_wait(&empty[s], ((cnt / nstage) & 1u) ^ 1u)) {
+          const int s = rp.s;
+          if (!mbar_wait(&empty[s], rp.ph ^ 1u)) {
             *s_abort = 1;
             break;
           }
@@ -350,13 +368,14 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
               tma_load_2d(st_x + q * XCOLS * kLine, &a.tm_x, xb0 + q * kLine, it.xrow0 + c0, &full[s], pol_x);
           }
           ++cnt;
+          rp.next();
         }
         item = next_item;
       }
       // end of work: one more stage whose header says so
       if (dynamic && !*s_abort) {
-        const int s = cnt % nstage;
-        if (mbar_wait(&empty[s], ((cnt / nstage) & 1u) ^ 1u)) {
+        const int s = rp.s;
+        if (mbar_wait(&empty[s], rp.ph ^ 1u)) {
           s_hdr[s] = -1;
           mbar_arrive(&full[s]);
           ++cnt;
@@ -396,20 +415,21 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
                                  : 0u;
   // the owned row inside its scale stage (gate rows of the stage's warps, then up rows)
   const int s_wl = warp % slot_warps;
+  const int s_slot = warp / slot_warps;  // the scale stage that carries this warp's rows
   // (half items own two rows per quad: lanes c and c+2 hold the same one)
   const int s_row = kHalf ? (kGateUp ? ((c & 1) ? kWarpRows * slot_warps : 0) + kWarpRows * s_wl + g
                                      : kWarpRows * s_wl + g + 8 * (c & 1))
                           : (kGateUp ? ((c >> 1) ? kWarpRows * slot_warps : 0) + kWarpRows * s_wl + g + 8 * (c & 1)
                                      : kWarpRows * s_wl + 16 * (c >> 1) + g + 8 * (c & 1));
-  uint32_t cnt = 0;
+  RingPos rc{0, 0u, nstage};
   const uint32_t stage0 = smem_u32(s_stage);
   for (int item = blockIdx.x;; item += gridDim.x) {
     if (dynamic) {
       // the item's first stage names it (or the end of work); the loops
       // below wait on it again: that phase is complete and cannot move on
       // before this warp releases the stage
-      const int s = cnt % nstage;
-      if (*s_abort || !mbar_wait(&full[s], (cnt / nstage) & 1u)) {
+      const int s = rc.s;
+      if (*s_abort || !mbar_wait(&full[s], rc.ph)) {
         *s_abort = 1;
         break;
       }
@@ -429,12 +449,12 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
     const int ng_act = ceil_div(ncols, 8);
     // --------------------------------------------- block scales -> TMEM
     for (int j = 0; j < n_sslots; ++j) {
-      const int s = cnt % nstage;
-      if (*s_abort || !mbar_wait(&full[s], (cnt / nstage) & 1u)) {
+      const int s = rc.s;
+      if (*s_abort || !mbar_wait(&full[s], rc.ph)) {
         *s_abort = 1;
         break;
       }
-      if (active && ncols > 0 && warp / slot_warps == j) {
+      if (active && ncols > 0 && s_slot == j) {
         const uint32_t ra = stage0 + s * STAGE_BYTES + s_row * srow;
         for (int cb = 0; cb < a.tmem_cols; cb += 4) {
           uint32_t v[4];
@@ -456,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
-      ++cnt;
+      rc.next();
     }
     if (*s_abort) break;
     float acc[NG][kMT][4];
@@ -481,14 +501,14 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
         }
     }
     for (int ch = ch_lo; ch < ch_hi; ++ch) {
-      const int s = cnt % nstage;
+      const int s = rc.s;
       const bool work = active && ncols > 0;
       // this chunk's scales of the owned row (issued before the wait for the stage)
       uint32_t sv[4] = {0u, 0u, 0u, 0u};
       if constexpr (Tr::blk != 0) {
         if (work) tc::tmem_ld_cols<kCpc>(t_row + ch * kCpc, sv);
       }
-      if (*s_abort || !mbar_wait(&full[s], (cnt / nstage) & 1u)) {
+      if (*s_abort || !mbar_wait(&full[s], rc.ph)) {
         if constexpr (Tr::blk != 0) {
           if (work) tc::tmem_ld_wait<kCpc>(sv);
         }
@@ -655,7 +675,7 @@ __global__ void __launch_bounds__(kThreads, MINB) ffn_stream_kernel(const __grid
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
-      ++cnt;
+      rc.next();
     }
     if (*s_abort) break;
     // ------------------------------------------------- split K: slice sums
