@@ -36,6 +36,17 @@ import moe_inputs as mi  # noqa: E402
 METRIC = "MoE-layer tokens/s and achieved HBM GB/s (decode) / TFLOPS (prefill) vs B200 peak"
 SHAPE = mi.GPTOSS
 PROFILE_EVERY = 10
+
+
+def profile_every(steps):
+    """Which timed steps carry per-kernel CUDA events (every n-th, never the
+    first).  Events between launches stop a kernel from overlapping its
+    predecessor, which costs a layer of a few tokens ~30 us on the steps that
+    carry them, so long runs sample sparsely: every 50th step from 500 steps
+    (10+ samples), every 10th from 100, else every step."""
+    if steps >= 50 * PROFILE_EVERY:
+        return 5 * PROFILE_EVERY
+    return PROFILE_EVERY if steps >= 10 * PROFILE_EVERY else 1
 DEFAULT_TOKENS = {"tiny": 16, "gptoss_decode": 64, "mixtral_prefill": 4096, "kimi_decode": 128,
                   "offload_bank": 16, "mixtral_prefill_mxfp4": 4096, "mixtral_prefill_nvfp4": 4096,
                   "mixtral_prefill_int4": 4096}
@@ -317,7 +328,7 @@ def stored_traffic(workload, T):
 def launches_per_step(prof, steps):
     """Kernel launches in the timed region: the sampled steps' launch count per
     step times the number of steps."""
-    every = PROFILE_EVERY if steps >= 10 * PROFILE_EVERY else 1
+    every = profile_every(steps)
     sampled = len([i for i in range(steps) if i > 0 and i % every == 0])
     per_step = sum(v[0] for v in prof.values()) / max(sampled, 1)
     return int(round(per_step * steps))
@@ -391,12 +402,12 @@ def run_ours(args):
     barrier()
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    # per-kernel CUDA events on every PROFILE_EVERY-th step of the timed region
-    # (events between launches also stop a kernel from overlapping its
-    # predecessor, so they are sampled rather than put around every launch)
-    # sampled steps: every 10th of a long run, every step but the first of a
-    # short one (the first timed step is never sampled)
-    every = PROFILE_EVERY if args.steps >= 10 * PROFILE_EVERY else 1
+    # per-kernel CUDA events on a sample of the timed steps (profile_every:
+    # every 50th of a run of 500+ steps, every 10th from 100, every step but
+    # the first of a short one); events between launches also stop a kernel
+    # from overlapping its predecessor, so they are sampled rather than put
+    # around every launch
+    every = profile_every(args.steps)
     e0.record(stream)
     for i in range(args.steps):
         if not args.no_kernel_timing:
