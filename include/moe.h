@@ -87,7 +87,7 @@ extern "C" {
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1,     /* null pointer, bad shape, misaligned pointer */
-  MOE_ERR_UNSUPPORTED = 2,     /* valid but outside what this build handles */
+  MOE_ERR_UNSUPPORTED = 2,     /* valid but outside what the library handles */
   MOE_ERR_CUDA = 3,            /* a CUDA runtime call or launch failed */
   MOE_ERR_OOM = 4,             /* cache allocation failed */
   MOE_ERR_CACHE_PINNED_FULL = 5, /* every slot of a layer is protected */
