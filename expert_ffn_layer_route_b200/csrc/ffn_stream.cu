@@ -888,8 +888,10 @@ cudaError_t launch_ffn_stream(int F, bool gate_up, FfnArgs a, const FfnPointers&
   // next K chunk reads, and marking them evict-first let L2 drop those halves
   // before that (DRAM reads 1.125 vs 1.042 GB per stage-1 launch; stage 1
   // 229 vs 204 us at T=64).  MOE_FFN_NG / MOE_FFN_MINB / MOE_W_L2FIRST
-  // override the choices for tuning.
-  int ng = (T <= 8 || (a.n_shared == 0 && (int64_t)T * a.k < 4LL * a.E)) ? 1 : 2;
+  // override the choices for tuning.  Batches of up to 16 tokens take one
+  // group even with shared experts (Kimi-shaped layer, T=16: 372 vs 384 us
+  // per layer; T=32: 564 vs 559 us, so two groups from there).
+  int ng = (T <= 16 || (a.n_shared == 0 && (int64_t)T * a.k < 4LL * a.E)) ? 1 : 2;
   // With one column group a block fits in a third of an SM (two stages of
   // 36 KB, 72 registers a thread): 24 consumer warps per SM hide more of the
   // decode's dependency latency than 16 (gpt-oss T=64: stage 1 at 0.77 vs 0.74
