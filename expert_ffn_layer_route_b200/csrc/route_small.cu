@@ -151,15 +151,23 @@ __global__ void __launch_bounds__(kRouterThreads) route_prep_small_kernel(const 
   for (int i = tid; i < R; i += kRouterThreads) s_rl[i] = rtok0[i];
   __syncthreads();
   cluster.barrier_arrive();
-  // one warp per row
+  // one CTA per row when the rows fit the cluster, else one warp per row
+  // (both group sizes give the same row: see prep_row)
   const int RT = R + a.n_shared * T;
-  const int nwarps = csize * (kRouterThreads / 32);
-  for (int r = rank * (kRouterThreads / 32) + warp; r < RT; r += nwarps) {
+  auto row_src = [&](int r) -> const __nv_bfloat16* {
     const int srow = r < R ? s_rl[r] : (r - R) % T;
-    const bool have = (unsigned)srow < (unsigned)T;  // a dropped pair's row has no source: zeros
-    prep_row<kMode, true>(have ? a.x + (size_t)srow * a.d : nullptr, a.d,
-                          static_cast<uint8_t*>(a.xperm) + (size_t)r * a.d * 2, a.xexp ? a.xexp + r : nullptr,
-                          a.gbias ? a.gbias + (size_t)r * (a.d / 128) : nullptr, tid & 31, 32, nullptr);
+    return (unsigned)srow < (unsigned)T ? a.x + (size_t)srow * a.d : nullptr;  // a dropped pair's row: zeros
+  };
+  auto row_dst = [&](int r) { return static_cast<uint8_t*>(a.xperm) + (size_t)r * a.d * 2; };
+  if (RT <= csize) {
+    if (rank < RT)
+      prep_row<kMode>(row_src(rank), a.d, row_dst(rank), a.xexp ? a.xexp + rank : nullptr,
+                      a.gbias ? a.gbias + (size_t)rank * (a.d / 128) : nullptr, tid, kRouterThreads, s_red);
+  } else {
+    const int nwarps = csize * (kRouterThreads / 32);
+    for (int r = rank * (kRouterThreads / 32) + warp; r < RT; r += nwarps)
+      prep_row<kMode, true>(row_src(r), a.d, row_dst(r), a.xexp ? a.xexp + r : nullptr,
+                            a.gbias ? a.gbias + (size_t)r * (a.d / 128) : nullptr, tid & 31, 32, nullptr);
   }
   cluster.barrier_wait();  // CTA 0's shared memory stays until every CTA has read it
 }
