@@ -42,6 +42,11 @@ constexpr int kSmallMaxT = 8;
 constexpr int kSmallMaxPairs = 64;
 // logits per router tile: 32 experts for one token, 4 for eight
 constexpr int kSmallTileLogits = 32;
+// experts per router tile for kTok tokens: at most 16, so that a CTA's slice
+// of 128 experts / 8 CTAs fills its tile without padding columns
+__host__ __device__ constexpr int small_tile_experts(int tok) {
+  return kSmallTileLogits / tok < 16 ? kSmallTileLogits / tok : 16;
+}
 
 struct RouteSmallArgs {
   const __nv_bfloat16* x;
@@ -78,7 +83,7 @@ __global__ void __launch_bounds__(kRouterThreads) route_prep_small_kernel(const 
   const int csize = (int)cluster.num_blocks();
   const int tid = threadIdx.x, warp = tid >> 5;
   extern __shared__ float smem_f[];
-  constexpr int kSmallExp = kSmallTileLogits / kTok;  // experts per router tile
+  constexpr int kSmallExp = small_tile_experts(kTok);  // experts per router tile
   float* s_part = smem_f;                      // [8 * kSmallTileLogits]
   float* s_red = s_part + 8 * kSmallTileLogits;  // [8]
   float* s_all = s_red + 8;                    // [kTok][E], filled on CTA 0
@@ -255,7 +260,7 @@ cudaError_t launch_small_mode(int mode, const RouteSmallArgs& a, cudaStream_t st
 }  // namespace
 
 // Used by default where one launch beats the four it replaces: batches of at
-// most 4 tokens whose router fits one tile per CTA (at most 32 / tile-tokens
+// most 4 tokens whose router fits one tile per CTA (at most min(16, 32 / tile-tokens)
 // experts per CTA of 8).  Measured on B200, the gpt-oss-shaped layer (128
 // experts, d = 2880) at T = 1 takes 52.5-54.8 us per layer fused vs 54.5-56.2
 // unfused; the Kimi-shaped layer (384 experts, d = 7168) runs its router
@@ -273,7 +278,7 @@ bool route_prep_small_supported(const moe_layer_desc& d) {
   }
   const int tok = d.T > 4 ? 8 : (d.T > 2 ? 4 : d.T);
   const int e_per_cta = ((ceil_div(d.n_experts, 8) + 3) / 4) * 4;
-  return fits && d.T <= 4 && e_per_cta <= kSmallTileLogits / tok;
+  return fits && d.T <= 4 && e_per_cta <= small_tile_experts(tok);
 }
 
 cudaError_t launch_route_prep_small(const moe_layer_desc& dsc, const void* x, const void* wr, const float* bias,
