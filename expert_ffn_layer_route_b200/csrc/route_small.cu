@@ -5,16 +5,18 @@
 // latency, not on bytes (the router, top-k, permutation and activation-prep
 // kernels each read a few KB to MB).  This kernel does all four as one
 // thread-block cluster:
-//   1. every CTA computes the router logits of its slice of the experts for
+//   1. every CTA brings its slice of the router weights into L2 before the
+//      dependent-launch wait, then computes the logits of its experts for
 //      all T tokens (the router tile of the standalone router kernel: the
-//      same fp32 summation tree, so the same logits);
-//   2. CTA 0 gathers the slices through distributed shared memory, selects
-//      each token's top-k with renormalised softmax gates (one warp per
-//      token, the standalone top-k routine) and forms the stable per-expert
-//      permutation (offsets, row of each (token, slot) pair, token of each
-//      row; rows of one expert in ascending token order);
-//   3. every CTA writes its share of the activation rows in expert order in
-//      the grouped FFN's input format (the standalone prep routine).
+//      same fp32 summation tree, so the same logits) and stores them into
+//      CTA 0's shared memory through distributed shared memory;
+//   2. CTA 0 selects each token's top-k with renormalised softmax gates (one
+//      warp per token, the standalone top-k routine) and forms the stable
+//      per-expert permutation by counting (offsets, row of each (token, slot)
+//      pair, token of each row; rows of one expert in ascending token order);
+//   3. the activation rows in expert order, in the grouped FFN's input format
+//      (the standalone prep routine): one CTA per row when the rows fit the
+//      cluster, else one warp per row.
 // The steps are ordered by cluster barriers, which the hardware schedules
 // together, so no counter or flag is polled.  The router step follows "a
 // router that picks a few of them per token" ("Mixture of experts VRAM:
