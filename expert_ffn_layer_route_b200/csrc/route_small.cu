@@ -229,8 +229,16 @@ cudaError_t launch_small(RouteSmallArgs a, cudaStream_t st) {
       (void)cudaGetLastError();
       continue;
     }
-    static std::atomic<int> fits16{-1};  // the occupancy answer, asked once per kernel
-    if (fits16.load() < 0) {
+    // the occupancy answer, asked once per kernel and device
+    constexpr int kMaxDev = 64;
+    static std::atomic<int> fits16_dev[kMaxDev];  // 0: not asked, 1: no, 2: yes
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+      (void)cudaGetLastError();
+      dev = 0;
+    }
+    std::atomic<int>& fits16 = fits16_dev[dev];
+    if (fits16.load() == 0) {
       cfg.gridDim = dim3(csize);
       cfg.dynamicSmemBytes = smem;
       attr[0].val.clusterDim.x = csize;
@@ -238,9 +246,9 @@ cudaError_t launch_small(RouteSmallArgs a, cudaStream_t st) {
       int n_clusters = 0;
       const bool ok = cudaOccupancyMaxActiveClusters(&n_clusters, kern, &cfg) == cudaSuccess && n_clusters > 0;
       if (!ok) (void)cudaGetLastError();
-      fits16.store(ok ? 1 : 0);
+      fits16.store(ok ? 2 : 1);
     }
-    if (fits16.load() == 1) break;
+    if (fits16.load() == 2) break;
   }
   cfg.gridDim = dim3(csize);
   cfg.dynamicSmemBytes = smem;
